@@ -1,0 +1,197 @@
+/*
+ * moe_b200.h -- C ABI of the B200 (sm_100a) DeepSeekMoE layer forward.
+ *
+ * The layer (sources, by page title and section):
+ *   [report-walkthrough] "DeepSeek-V3 technical report" walkthrough (2kiu.com),
+ *       section 3.2 (sigmoid affinities, bias-ranked top-K, gates from s,
+ *       batch-level bias update), section 3.4 (node-limited routing),
+ *       section 4.3 (FP8 block scaling, high-precision accumulation);
+ *   [repro-guide] "From technical report to a runnable config" (lpnh.cn),
+ *       section 3 (num_experts 256, 1 shared, top-8, moe_intermediate 2048,
+ *       norm_topk_prob, routed_scaling_factor 2.5, e4m3, 1x128 input tiles,
+ *       128x128 weight blocks, moe_gating kept in high precision);
+ *   [infra-answer] Zhihu answer on DeepSeek-V3's infrastructure: E4M3
+ *       throughout, per-tile/per-group scales, partial-sum promotion.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library never allocates or frees memory.  Row-major everywhere;
+ *     weights are [N, K] with K contiguous ("K-major").
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous and stream-ordered, keep no state
+ *     between calls, and are safe to call from several host threads.
+ *   - Host-side argument checks run before any launch and return
+ *     MOE_ERR_INVALID_ARG (bad sizes, NULL or misaligned pointers) or
+ *     MOE_ERR_UNSUPPORTED (valid but outside what the kernels implement).
+ *     A launch failure returns MOE_ERR_CUDA.  Zero-size work returns MOE_OK
+ *     without launching.
+ *   - `status`, where present, is an optional device int32 that kernels
+ *     OR MOE_FLAG_* bits into (never cleared by the library); NULL skips it.
+ *   - Pointers to packed 16-byte vectors (bf16 rows, e4m3 rows, scales)
+ *     must be 16-byte aligned.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Problem statement of one layer, as the pages state it: T tokens, hidden
+ * size H, E routed experts, top-K, n_group expert groups of which
+ * topk_group are kept per token (the node limit of [report-walkthrough]
+ * section 3.4), expert intermediate size I and routed_scaling_factor
+ * ([repro-guide] section 3). */
+typedef struct moe_dims {
+    int32_t T, H, E, K, n_group, topk_group, I;
+    float routed_scaling_factor;
+} moe_dims;
+
+enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,
+    MOE_ERR_UNSUPPORTED = 2,
+    MOE_ERR_WORKSPACE = 3,
+    MOE_ERR_CUDA = 4
+};
+
+/* Bits kernels OR into the optional device status word. */
+enum moe_flag {
+    MOE_FLAG_NONFINITE = 1,  /* a quantised tile held NaN/Inf: codes 0x7F, scale NaN */
+    MOE_FLAG_BAD_INDEX = 2,  /* an expert index outside [0, E): entry skipped          */
+    MOE_FLAG_TIMEOUT = 4,    /* a bounded on-device wait gave up; outputs undefined     */
+    MOE_FLAG_BAD_OFFSETS = 8 /* group offsets not monotone or beyond m_capacity         */
+};
+
+/* GEMM epilogues. */
+enum moe_epilogue {
+    MOE_EPI_BF16 = 0,          /* C bf16 [M, N]                                      */
+    MOE_EPI_F32 = 1,           /* C fp32 [M, N]                                      */
+    MOE_EPI_SWIGLU_REQUANT = 2 /* N = 2I: C e4m3 [M, I] codes, sC fp32 [M, I/128]      */
+};
+
+/* Human-readable name of a moe_status value.  Static string, never NULL. */
+const char *moe_status_string(int status);
+
+/* Library ABI version (increments on any signature change). */
+int moe_abi_version(void);
+
+/* Bytes of scratch `ws` that moe_route and moe_permute need for `dims`
+ * (the larger of the two).  ws must be 256-byte aligned. */
+size_t moe_workspace_size(const moe_dims *dims);
+
+/* Activation quantisation, one scale per 1x128 tile ([report-walkthrough]
+ * section 4.3; [repro-guide] section 3 input_quant_granularity
+ * tile_wise_1x128, format e4m3).  For each row r and tile j:
+ *   amax = max |x[r, 128j .. 128j+127]|
+ *   scales[r, j] = amax == 0 ? 1 : fp32(amax / 448)
+ *   q[r, c] = e4m3_rne_satfinite(fp32(x[r, c] / scales[r, j]))
+ * A tile holding NaN/Inf gets codes 0x7F, scale NaN and MOE_FLAG_NONFINITE.
+ *   x      bf16 [rows, cols], cols % 128 == 0
+ *   q      e4m3 codes uint8 [rows, cols]
+ *   scales fp32 [rows, cols/128]                                              */
+int fp8_quant_1x128(const void *x, int64_t rows, int64_t cols, uint8_t *q, float *scales,
+                    int32_t *status, void *stream);
+
+/* Weight quantisation, one scale per 128x128 block ([repro-guide] section 3
+ * weight_quant_granularity block_wise_128x128; [infra-answer]).  Same rule
+ * as fp8_quant_1x128 with the block in place of the tile.  A setup step.
+ *   w      bf16 [batch, rows, cols], rows % 128 == 0, cols % 128 == 0
+ *   q      uint8 [batch, rows, cols]
+ *   scales fp32 [batch, rows/128, cols/128]                                   */
+int fp8_quant_128x128(const void *w, int64_t batch, int64_t rows, int64_t cols, uint8_t *q,
+                      float *scales, int32_t *status, void *stream);
+
+/* Router ([report-walkthrough] sections 3.2 and 3.4; gating kept in fp32 per
+ * [repro-guide] section 3 keep_bf16 moe_gating):
+ *   s = sigmoid(x W_r^T + router_offset)      fp32 accumulation
+ *   r = s + e_bias (one fp32 add); group score = fp32 sum of the top
+ *   min(2, E/n_group) r in each of n_group groups; keep the topk_group best
+ *   groups; topk_idx = top-K of r over the kept experts, in descending r,
+ *   ties to the lower index (groups and experts alike);
+ *   topk_w[t,k] = fp32((rho * s_k) / sum_j s_j) evaluated in float64.
+ *   x             bf16 [T, H]
+ *   w_router      fp32 [E, H]
+ *   e_bias        fp32 [E]
+ *   router_offset fp32 [E] additive logit offset, or NULL
+ *   topk_idx      int32 [T, K];  topk_w fp32 [T, K]
+ *   scores        fp32 [T, E] output of s, or NULL (then ws holds it)
+ * Limits: E <= 1024, E % n_group == 0, n_group <= 32, K <= 32,
+ * topk_group * E / n_group >= K, H % 128 == 0.                                 */
+int moe_route(const moe_dims *dims, const void *x, const float *w_router, const float *e_bias,
+              const float *router_offset, int32_t *topk_idx, float *topk_w, float *scores,
+              void *ws, size_t ws_bytes, int32_t *status, void *stream);
+
+/* The selection half of moe_route alone, on given affinities s fp32 [T, E]. */
+int moe_route_select(const moe_dims *dims, const float *scores, const float *e_bias,
+                     int32_t *topk_idx, float *topk_w, void *stream);
+
+/* Dispatch into per-expert segments (the token-to-expert step of
+ * [report-walkthrough] sections 3.2 and 4.1; no token is dropped, section
+ * 3.4).  A stable counting sort of the T*K (token, slot) pairs by expert:
+ *   expert_load[e]    = #pairs routed to e                     int32 [E]
+ *   expert_offsets[e] = exclusive prefix of expert_load        int32 [E+1]
+ *   rows offsets[e] .. offsets[e+1]-1 hold expert e's pairs in ascending
+ *   token order; tok_of[row] = token, row_of[t*K + k] = row    int32 [T*K]
+ *   aq[row, :] = xq[tok_of[row], :]  (e4m3 [T*K, H]),
+ *   as[row, :] = xs[tok_of[row], :]  (fp32 [T*K, H/128]);
+ * xq/xs/aq/as may all be NULL to build the maps only.  An index outside
+ * [0, E) raises MOE_FLAG_BAD_INDEX and that pair gets row_of = -1.         */
+int moe_permute(const moe_dims *dims, const int32_t *topk_idx, const uint8_t *xq, const float *xs,
+                int32_t *expert_load, int32_t *expert_offsets, int32_t *tok_of, int32_t *row_of,
+                uint8_t *aq, float *as, void *ws, size_t ws_bytes, int32_t *status, void *stream);
+
+/* Grouped FP8 GEMM with block scales, promoted every 128 of K
+ * ([report-walkthrough] section 4.3; [infra-answer]: the tile/block scales
+ * have no hardware support, so partial sums are promoted).  For group g,
+ * rows m in [group_offsets[g], group_offsets[g+1]):
+ *   C[m, n] = sum_kb sA[m, kb] * sB[g, n/128, kb] *
+ *             sum_{k in kb} e4m3(A[m, k]) * e4m3(B[g, n, k])
+ * with fp32 accumulation of each 128-wide partial and of the promotion.
+ *   group_offsets  device int32 [G+1], non-decreasing, last <= m_capacity
+ *   A   e4m3 [m_capacity, K];  sA fp32 [m_capacity, K/128]
+ *   B   e4m3 [G, N, K];        sB fp32 [G, N/128, K/128]
+ *   MOE_EPI_BF16 / MOE_EPI_F32: C [m_capacity, N] (rows outside every
+ *   group are not written).
+ *   MOE_EPI_SWIGLU_REQUANT: B rows 0..I-1 are the gate and I..2I-1 the up
+ *   projection (N = 2I); act = silu(g) * u in fp32, then the 1x128 rule of
+ *   fp8_quant_1x128: C e4m3 [m_capacity, I], sC fp32 [m_capacity, I/128].
+ * Limits: K % 128 == 0, N % 128 == 0 (SwiGLU: I % 128 == 0), G <= 4096.    */
+int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets, int64_t m_capacity,
+                                 int64_t N, int64_t K, const uint8_t *A, const float *sA,
+                                 const uint8_t *B, const float *sB, int32_t epilogue, void *C,
+                                 float *sC, int32_t *status, void *stream);
+
+/* SwiGLU and 1x128 requantisation of a given fp32 [M, 2I] gate|up matrix
+ * (the GEMM epilogue's arithmetic as a stand-alone call; SwiGLU named in
+ * [infra-answer], expert intermediate I per [arch-overview]
+ * "DeepSeek-V3 MoE architecture and FP8 training" (0539edu.com)):
+ *   act = (g / (1 + exp(-g))) * u   in fp32;  q, s as in fp8_quant_1x128.
+ *   q uint8 [M, I];  s fp32 [M, I/128]                                        */
+int swiglu_requant(const float *gu, int64_t M, int64_t I, uint8_t *q, float *s, int32_t *status,
+                   void *stream);
+
+/* Gated combine ([report-walkthrough] section 3.2: y = sum_j gate_j *
+ * ffn_{idx_j}(h)) plus the shared expert:
+ *   out[t] = sum_k topk_w[t,k] * yperm[row_of[t*K+k]] + yshared[t]
+ * summed in fp32 in k order (shared last), stored as bf16 and optionally fp32.
+ *   yperm bf16 [T*K, H]; yshared bf16 [T, H] or NULL; out bf16 [T, H];
+ *   out_f32 fp32 [T, H] or NULL.  Pairs with row_of < 0 are skipped.          */
+int moe_combine(const moe_dims *dims, const void *yperm, const int32_t *row_of,
+                const float *topk_w, const void *yshared, void *out, float *out_f32, void *stream);
+
+/* Auxiliary-loss-free bias update ([report-walkthrough] section 3.2; rate
+ * expert_bias_update_rate 0.001 in [repro-guide] section 3):
+ *   e_bias[e] += gamma * sign(T*K/E - expert_load[e]),  sign(0) = 0,
+ * one fp32 addition per expert; the comparison is exact (T*K vs E*load).   */
+int moe_bias_update(int32_t E, int64_t T, int32_t K, float gamma, const int32_t *expert_load,
+                    float *e_bias, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,165 @@
+"""ctypes binding of libmoe_b200.so: argument marshalling only.
+
+Every function here has the name of its C entry point (include/moe_b200.h),
+takes torch tensors (device memory owned by the caller) or None, passes their
+data pointers and the current CUDA stream, and raises MoEError on a non-zero
+return code.  No arithmetic of the layer happens in Python.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA = range(5)
+MOE_FLAG_NONFINITE, MOE_FLAG_BAD_INDEX, MOE_FLAG_TIMEOUT, MOE_FLAG_BAD_OFFSETS = 1, 2, 4, 8
+MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_REQUANT = 0, 1, 2
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {code}: {status_string(code)}")
+        self.code = code
+
+
+class MoeDims(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("K", ctypes.c_int32), ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32),
+                ("I", ctypes.c_int32), ("routed_scaling_factor", ctypes.c_float)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m sparse_moe_layer_group_b200.build` "
+            "(there is no fallback path)")
+    return ctypes.CDLL(LIB_PATH)
+
+
+_lib = _load()
+
+_P, _I32, _I64, _F, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+_DIMS = ctypes.POINTER(MoeDims)
+
+_SIGS = {
+    "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "moe_abi_version": (ctypes.c_int, []),
+    "moe_workspace_size": (_SZ, [_DIMS]),
+    "fp8_quant_1x128": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P]),
+    "fp8_quant_128x128": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P]),
+    "moe_route": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
+    "moe_route_select": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P]),
+    "moe_permute": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
+    "fp8_grouped_gemm_blockscaled": (ctypes.c_int, [_I32, _P, _I64, _I64, _I64, _P, _P, _P, _P, _I32,
+                                                    _P, _P, _P, _P]),
+    "swiglu_requant": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P]),
+    "moe_combine": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_bias_update": (ctypes.c_int, [_I32, _I64, _I32, _F, _P, _P, _P]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+
+def status_string(code: int) -> str:
+    return _lib.moe_status_string(int(code)).decode()
+
+
+def abi_version() -> int:
+    return int(_lib.moe_abi_version())
+
+
+def dims(T, H, E, K, n_group, topk_group, I, rho) -> MoeDims:
+    return MoeDims(int(T), int(H), int(E), int(K), int(n_group), int(topk_group), int(I), float(rho))
+
+
+def workspace_size(d: MoeDims) -> int:
+    return int(_lib.moe_workspace_size(ctypes.byref(d)))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn: str, rc: int):
+    if rc != MOE_OK:
+        raise MoEError(fn, rc)
+
+
+def fp8_quant_1x128(x, q, scales, status=None, stream=None):
+    rows, cols = x.shape
+    _check("fp8_quant_1x128", _lib.fp8_quant_1x128(_ptr(x), rows, cols, _ptr(q), _ptr(scales),
+                                                   _ptr(status), _stream(stream)))
+
+
+def fp8_quant_128x128(w, q, scales, status=None, stream=None):
+    if w.dim() == 2:
+        batch, (rows, cols) = 1, w.shape
+    else:
+        batch, rows, cols = w.shape
+    _check("fp8_quant_128x128", _lib.fp8_quant_128x128(_ptr(w), batch, rows, cols, _ptr(q), _ptr(scales),
+                                                       _ptr(status), _stream(stream)))
+
+
+def moe_route(d, x, w_router, e_bias, router_offset, topk_idx, topk_w, scores=None, ws=None,
+              status=None, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("moe_route", _lib.moe_route(ctypes.byref(d), _ptr(x), _ptr(w_router), _ptr(e_bias),
+                                       _ptr(router_offset), _ptr(topk_idx), _ptr(topk_w), _ptr(scores),
+                                       _ptr(ws), ws_bytes, _ptr(status), _stream(stream)))
+
+
+def moe_route_select(d, scores, e_bias, topk_idx, topk_w, stream=None):
+    _check("moe_route_select", _lib.moe_route_select(ctypes.byref(d), _ptr(scores), _ptr(e_bias),
+                                                     _ptr(topk_idx), _ptr(topk_w), _stream(stream)))
+
+
+def moe_permute(d, topk_idx, xq, xs, expert_load, expert_offsets, tok_of, row_of, aq, as_, ws,
+                status=None, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("moe_permute", _lib.moe_permute(ctypes.byref(d), _ptr(topk_idx), _ptr(xq), _ptr(xs),
+                                           _ptr(expert_load), _ptr(expert_offsets), _ptr(tok_of),
+                                           _ptr(row_of), _ptr(aq), _ptr(as_), _ptr(ws), ws_bytes,
+                                           _ptr(status), _stream(stream)))
+
+
+def fp8_grouped_gemm_blockscaled(G, group_offsets, m_capacity, N, K, A, sA, B, sB, epilogue, C, sC=None,
+                                 status=None, stream=None):
+    _check("fp8_grouped_gemm_blockscaled", _lib.fp8_grouped_gemm_blockscaled(
+        int(G), _ptr(group_offsets), int(m_capacity), int(N), int(K), _ptr(A), _ptr(sA), _ptr(B), _ptr(sB),
+        int(epilogue), _ptr(C), _ptr(sC), _ptr(status), _stream(stream)))
+
+
+def swiglu_requant(gu, q, s, status=None, stream=None):
+    M, two_i = gu.shape
+    _check("swiglu_requant", _lib.swiglu_requant(_ptr(gu), M, two_i // 2, _ptr(q), _ptr(s), _ptr(status),
+                                                 _stream(stream)))
+
+
+def moe_combine(d, yperm, row_of, topk_w, yshared, out, out_f32=None, stream=None):
+    _check("moe_combine", _lib.moe_combine(ctypes.byref(d), _ptr(yperm), _ptr(row_of), _ptr(topk_w),
+                                           _ptr(yshared), _ptr(out), _ptr(out_f32), _stream(stream)))
+
+
+def moe_bias_update(E, T, K, gamma, expert_load, e_bias, stream=None):
+    _check("moe_bias_update", _lib.moe_bias_update(int(E), int(T), int(K), float(gamma), _ptr(expert_load),
+                                                   _ptr(e_bias), _stream(stream)))

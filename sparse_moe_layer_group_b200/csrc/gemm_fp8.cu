@@ -1,0 +1,547 @@
+// Grouped FP8 (E4M3) GEMM with 1x128 / 128x128 block scales, promoted every 128
+// of K, on the sm_100a tensor cores (tcgen05 + TMEM, operands staged by TMA).
+//
+// What it computes ("DeepSeek-V3 technical report" walkthrough (2kiu.com),
+// section 4.3; the Zhihu infrastructure answer on DeepSeek-V3: per-tile 1x128
+// activation scales and per-block 128x128 weight scales are not supported by the
+// tensor cores, so the product is formed as partial sums that are promoted):
+//   C[m, n] = sum_kb  sA[m, kb] * sB[g, n/128, kb] * P_kb[m, n],
+//   P_kb    = sum_{k in kb} e4m3(A[m, k]) * e4m3(B[g, n, k])   (fp32, tensor core)
+// for the rows m of group g.  Each 128-wide K block is accumulated by the tensor
+// core into a fresh TMEM buffer; the epilogue warps read it (tcgen05.ld), scale it
+// and add it to fp32 registers.  Two TMEM buffers (2 x 256 columns) let the
+// tensor core run block kb+1 while the epilogue promotes block kb.
+//
+// CTA organisation (persistent: one CTA per SM, 384 threads):
+//   warp 0        TMA producer: A tile 128x128 B + B tile 256x128 B per stage
+//   warp 1        TMEM allocator and MMA issuer (one elected lane)
+//   warps 2-3     idle (complete warpgroup 0 for setmaxnreg)
+//   warps 4-11    epilogue: warp w reads TMEM lanes 32*(w%4).., the two
+//                 warpgroups split the 256 accumulator columns
+// Tiles: 128 rows x 256 columns; the tile list (group-major, then N tile, then M
+// tile so that consecutive CTAs share a weight tile through L2) is derived on the
+// device from group_offsets, so no host synchronisation is needed.
+//
+// No cluster launch and no multicast: every CTA loads its own tiles.  Every wait
+// is bounded (2 s); on expiry the CTA raises MOE_FLAG_TIMEOUT, drains its own
+// outstanding TMA loads and MMAs, frees its TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+
+namespace moe {
+namespace gg {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;          // bytes == e4m3 elements == one 128B swizzle row
+constexpr int STAGES = 4;
+constexpr uint32_t A_BYTES = BM * BK;
+constexpr uint32_t B_HALF = 128 * BK;
+constexpr uint32_t B_BYTES = BN * BK;
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int THREADS = 384;
+constexpr int EPI_THREADS = 256;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int MAX_G = 4096;
+constexpr uint64_t WAIT_NS = 2000000000ull;
+constexpr int LAUNCH_REGS = 168;   // 384 threads x 168 = 128 x 40 + 256 x 232
+
+// shared memory map (offsets from a 1024-aligned base)
+constexpr uint32_t OFF_STAGES = 0;
+constexpr uint32_t OFF_BARS = STAGES * STAGE_BYTES;                // 196608
+constexpr uint32_t OFF_MISC = OFF_BARS + 128;                      // tmem holder, abort, n_tiles, bad
+constexpr uint32_t OFF_RED = OFF_MISC + 32;                        // [2 parity][2 half][128] fp32
+constexpr uint32_t OFF_MSTART = OFF_RED + 2 * 2 * 128 * 4;         // int32 [MAX_G + 1]
+constexpr uint32_t SMEM_USED = OFF_MSTART + (MAX_G + 1) * 4;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;                  // + alignment slack
+
+// instruction descriptor: D fp32, A/B e4m3, K-major both, N = 256, M = 128
+constexpr uint32_t IDESC = (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+                           (static_cast<uint32_t>(BM >> 4) << 24);
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: false when another role aborted (unless drain is set: the
+// end-of-kernel drains wait out their own 2 s even after an abort) or the 2 s
+// budget ran out.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                       int32_t *status, bool drain = false) {
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try(bar, parity)) return true;
+        if ((n & 63u) == 0) {
+            if (!drain && *abort_flag) return false;
+            if (globaltimer() - t0 > WAIT_NS) {
+                *abort_flag = 1;
+                set_flag(status, MOE_FLAG_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *tm, int32_t c0, int32_t c1,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *tm, int32_t c0, int32_t c1,
+                                            int32_t c2, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// K-major operand in 128-byte-swizzled rows of 128 bytes, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+           (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+           (static_cast<uint64_t>(2) << 61);
+}
+
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(IDESC), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane; the wait sits in the
+// same asm statement so no use of r can be scheduled before the data arrive.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+struct Tile {
+    int g, m0, m_end, nt;
+};
+
+// Tile t -> (group, first row, group end, N tile).  Group g owns the tiles
+// [NT*mstart[g], NT*mstart[g+1]), ordered N-tile-major, M tile innermost.
+__device__ __forceinline__ Tile decode_tile(int t, const int32_t *mstart, int G, int NT,
+                                            const int32_t *__restrict__ offs) {
+    int lo = 0, hi = G;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (NT * mstart[mid] <= t) lo = mid; else hi = mid;
+    }
+    const int mcount = mstart[lo + 1] - mstart[lo];
+    const int local = t - NT * mstart[lo];
+    Tile r;
+    r.g = lo;
+    r.nt = local / mcount;
+    const int mt = local % mcount;
+    r.m0 = __ldg(offs + lo) + mt * BM;
+    r.m_end = __ldg(offs + lo + 1);
+    return r;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const int32_t *__restrict__ offs, int G, int64_t m_cap, int N, int K,
+                    const float *__restrict__ sA, const float *__restrict__ sB, int epi,
+                    void *__restrict__ C, float *__restrict__ sC, int32_t *status) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
+    const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
+    uint8_t *smem = smem_raw + pad;
+    const uint32_t sbase = raw_addr + pad;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t bar0 = sbase + OFF_BARS;
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
+    auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+    auto xchg_bar = [&](int p) { return bar0 + 8u * (2 * STAGES + 5 + p); };
+
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+    int *bad_flag = reinterpret_cast<int *>(smem + OFF_MISC + 8);
+    float *red = reinterpret_cast<float *>(smem + OFF_RED);
+    int32_t *mstart = reinterpret_cast<int32_t *>(smem + OFF_MSTART);
+
+    const bool swiglu = epi == MOE_EPI_SWIGLU_REQUANT;
+    const int I = N / 2;
+    const int NT = swiglu ? I / 128 : (N + BN - 1) / BN;
+    const int KB = K / BK;
+    const int NB = N / 128;
+
+    // ---- setup: per-group M-tile counts -> prefix; barriers; TMEM
+    if (threadIdx.x == 0) { *abort_flag = 0; *bad_flag = 0; }
+    __syncthreads();
+    for (int g = threadIdx.x; g < G; g += THREADS) {
+        const int a = __ldg(offs + g), b = __ldg(offs + g + 1);
+        if (b < a || a < 0 || static_cast<int64_t>(b) > m_cap) *bad_flag = 1;
+        mstart[g + 1] = b > a ? (b - a + BM - 1) / BM : 0;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        for (int base = 0; base < G; base += 32) {
+            const int g = base + lane;
+            int v = g < G ? mstart[g + 1] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += n;
+            }
+            if (g < G) mstart[g + 1] = v + carry;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+        if (lane == 0) mstart[0] = 0;
+    } else if (warp == 2 && lane == 0) {
+        for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
+        for (int b = 0; b < 2; ++b) { mbar_init(tfull_bar(b), 1); mbar_init(tempty_bar(b), EPI_THREADS); }
+        mbar_init(drain_bar, 1);
+        for (int p = 0; p < 2; ++p) mbar_init(xchg_bar(p), EPI_THREADS);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    } else if (warp == 3 && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+    }
+    if (warp == 1) {
+        __syncwarp();
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         sbase + OFF_MISC),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+    const int num_tiles = *bad_flag ? 0 : NT * mstart[G];
+    if (blockIdx.x == 0 && threadIdx.x == 0 && *bad_flag) set_flag(status, MOE_FLAG_BAD_OFFSETS);
+
+    __syncwarp();
+    if (warp < 4) {
+        // warpgroup 0 gives registers away to the two epilogue warpgroups
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;" ::: "memory");
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+                const Tile tl = decode_tile(t, mstart, G, NT, offs);
+                const int r0 = swiglu ? 128 * tl.nt : BN * tl.nt;
+                const int r1 = swiglu ? I + 128 * tl.nt : BN * tl.nt + 128;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, status)) { ok = false; break; }
+                    const uint32_t sa = sbase + OFF_STAGES + stage * STAGE_BYTES;
+                    mbar_expect_tx(full_bar(stage), STAGE_BYTES);
+                    tma_load_2d(sa, &tmA, kb * BK, tl.m0, full_bar(stage));
+                    tma_load_3d(sa + A_BYTES, &tmB, kb * BK, r0, tl.g, full_bar(stage));
+                    tma_load_3d(sa + A_BYTES + B_HALF, &tmB, kb * BK, r1, tl.g, full_bar(stage));
+                    ++issued;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // no TMA write may land after this CTA exits: wait for the last loads
+            const int tail = issued < STAGES ? issued : STAGES;
+            for (int i = 0; i < tail; ++i) {
+                if (stage == 0) { stage = STAGES - 1; phase ^= 1u; } else { --stage; }
+                mbar_wait(full_bar(stage), phase, abort_flag, status, true);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, kc = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+                for (int kb = 0; kb < KB; ++kb, ++kc) {
+                    const uint32_t buf = kc & 1u, use = kc >> 1;
+                    if (!mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
+                    if (!mbar_wait(full_bar(stage), phase, abort_flag, status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = sbase + OFF_STAGES + stage * STAGE_BYTES;
+                    const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sa + A_BYTES);
+                    const uint32_t d = tmem_base + buf * 256u;
+#pragma unroll
+                    for (int k = 0; k < BK / 32; ++k) mma_f8(d, ad + 2u * k, bd + 2u * k, k > 0 ? 1u : 0u);
+                    mma_commit(empty_bar(stage));
+                    mma_commit(tfull_bar(buf));
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // every MMA of this CTA has completed before TMEM is released
+            mma_commit(drain_bar);
+            mbar_wait(drain_bar, 0, abort_flag, status, true);
+        }
+    }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 232;" ::: "memory");
+        // ------------------------------------------------------ epilogue
+        const int q = warp & 3;               // TMEM lane quarter
+        const int half = (warp - 4) >> 2;     // column half of the 256-wide tile
+        const int row = q * 32 + lane;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+        uint32_t kc = 0, xphase0 = 0, xphase1 = 0;
+        int iter = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x, ++iter) {
+            const Tile tl = decode_tile(t, mstart, G, NT, offs);
+            const int64_t grow = static_cast<int64_t>(tl.m0) + row;
+            const bool row_ok = grow < m_cap;
+            const float *sa_row = sA + (row_ok ? grow : 0) * KB;
+            // per-chunk TMEM column and scale row of B
+            int nb0, nb1;
+            bool nb1_ok = true;
+            if (swiglu) { nb0 = tl.nt; nb1 = I / 128 + tl.nt; }
+            else { nb0 = 2 * tl.nt + half; nb1 = nb0; nb1_ok = nb0 < NB; }
+            const float *sb0 = sB + (static_cast<int64_t>(tl.g) * NB + (nb1_ok ? nb0 : 0)) * KB;
+            const float *sb1 = sB + (static_cast<int64_t>(tl.g) * NB + (nb1_ok ? nb1 : 0)) * KB;
+            float acc[128];
+#pragma unroll
+            for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+            for (int kb = 0; kb < KB; ++kb, ++kc) {
+                const float a_s = row_ok ? __ldg(sa_row + kb) : 0.0f;
+                const float s0 = nb1_ok ? __fmul_rn(a_s, __ldg(sb0 + kb)) : 0.0f;
+                const float s1 = nb1_ok ? __fmul_rn(a_s, __ldg(sb1 + kb)) : 0.0f;
+                const uint32_t buf = kc & 1u, use = kc >> 1;
+                if (!mbar_wait(tfull_bar(buf), use & 1u, abort_flag, status)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    // SwiGLU: chunks 0,1 gate columns 64*half + 32c; chunks 2,3 up columns 128 + 64*half + 32(c-2)
+                    // plain : chunk c columns 128*half + 32c
+                    const uint32_t col = swiglu ? (c < 2 ? 64u * half + 32u * c : 128u + 64u * half + 32u * (c - 2))
+                                                : 128u * half + 32u * c;
+                    uint32_t r[32];
+                    tmem_ld32(lane_base + buf * 256u + col, r);
+                    const float sc = (swiglu && c >= 2) ? s1 : s0;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) acc[32 * c + j] = fmaf(sc, __uint_as_float(r[j]), acc[32 * c + j]);
+                }
+                tc_fence_before();
+                mbar_arrive(tempty_bar(buf));
+            }
+            if (!ok) break;
+            const bool store_row = grow < tl.m_end;
+            if (!swiglu) {
+                const int64_t n0 = static_cast<int64_t>(tl.nt) * BN + 128 * half;
+                if (store_row && n0 < N) {
+                    if (epi == MOE_EPI_BF16) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(C) + grow * N + n0);
+#pragma unroll
+                        for (int v = 0; v < 16; ++v) {
+                            uint4 o;
+                            __nv_bfloat162 p0 = __floats2bfloat162_rn(acc[8 * v + 0], acc[8 * v + 1]);
+                            __nv_bfloat162 p1 = __floats2bfloat162_rn(acc[8 * v + 2], acc[8 * v + 3]);
+                            __nv_bfloat162 p2 = __floats2bfloat162_rn(acc[8 * v + 4], acc[8 * v + 5]);
+                            __nv_bfloat162 p3 = __floats2bfloat162_rn(acc[8 * v + 6], acc[8 * v + 7]);
+                            o.x = *reinterpret_cast<uint32_t *>(&p0);
+                            o.y = *reinterpret_cast<uint32_t *>(&p1);
+                            o.z = *reinterpret_cast<uint32_t *>(&p2);
+                            o.w = *reinterpret_cast<uint32_t *>(&p3);
+                            dst[v] = o;
+                        }
+                    } else {
+                        float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(C) + grow * N + n0);
+#pragma unroll
+                        for (int v = 0; v < 32; ++v)
+                            dst[v] = make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+                    }
+                }
+            } else {
+                // act = silu(g) * u on this thread's 64 columns, amax over the full
+                // 128-column tile via the partner warpgroup (same row, other half)
+                float amax = 0.0f;
+                bool fin = true;
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    acc[j] = swiglu_act(acc[j], acc[64 + j]);
+                    amax_step(acc[j], amax, fin);
+                }
+                const int p = iter & 1;
+                float *rp = red + p * 256;
+                rp[half * 128 + row] = fin ? amax : __int_as_float(0x7fc00000);
+                mbar_arrive(xchg_bar(p));
+                uint32_t &xph = p ? xphase1 : xphase0;
+                if (!mbar_wait(xchg_bar(p), xph, abort_flag, status)) { ok = false; break; }
+                xph ^= 1u;
+                const float mine = rp[half * 128 + row], other = rp[(half ^ 1) * 128 + row];
+                const bool finite = !isnan(mine) && !isnan(other);
+                const float sc = tile_scale(fmaxf(mine, other), finite);
+                if (store_row) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(C) + grow * I +
+                                                           128 * tl.nt + 64 * half);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int j = 16 * v + 4 * u;
+                            w[u] = static_cast<uint32_t>(quant_code(acc[j], sc, finite)) |
+                                   static_cast<uint32_t>(quant_code(acc[j + 1], sc, finite)) << 8 |
+                                   static_cast<uint32_t>(quant_code(acc[j + 2], sc, finite)) << 16 |
+                                   static_cast<uint32_t>(quant_code(acc[j + 3], sc, finite)) << 24;
+                        }
+                        dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                    if (half == 0) {
+                        sC[grow * (I / 128) + tl.nt] = sc;
+                        if (!finite) set_flag(status, MOE_FLAG_NONFINITE);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+static int prepare_kernel() {
+    static int state = 0;   // 0 unknown, 1 ready, 2 unsupported
+    if (state == 0) {
+        cudaFuncAttributes attr;
+        if (cudaFuncGetAttributes(&attr, grouped_gemm_kernel) != cudaSuccess) return MOE_ERR_CUDA;
+        // setmaxnreg moves registers inside the launch's allotment: the split
+        // 128 x 40 + 256 x 232 must equal 384 x (registers at launch)
+        if (attr.numRegs != LAUNCH_REGS) { state = 2; return MOE_ERR_UNSUPPORTED; }
+        if (cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(SMEM_BYTES)) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        state = 1;
+    }
+    return state == 1 ? MOE_OK : MOE_ERR_UNSUPPORTED;
+}
+
+}  // namespace gg
+}  // namespace moe
+
+using namespace moe;
+
+MOE_API int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets, int64_t m_capacity,
+                                         int64_t N, int64_t K, const uint8_t *A, const float *sA,
+                                         const uint8_t *B, const float *sB, int32_t epilogue, void *C,
+                                         float *sC, int32_t *status, void *stream) {
+    using namespace moe::gg;
+    if (G < 0 || m_capacity < 0 || N < 0 || K < 0) return MOE_ERR_INVALID_ARG;
+    if (N % 128 != 0 || K % 128 != 0) return MOE_ERR_INVALID_ARG;
+    if (epilogue != MOE_EPI_BF16 && epilogue != MOE_EPI_F32 && epilogue != MOE_EPI_SWIGLU_REQUANT)
+        return MOE_ERR_INVALID_ARG;
+    if (epilogue == MOE_EPI_SWIGLU_REQUANT && (N % 256 != 0 || !sC)) return MOE_ERR_INVALID_ARG;
+    if (G == 0 || m_capacity == 0 || N == 0) return MOE_OK;
+    if (K == 0) return MOE_ERR_UNSUPPORTED;   // an empty reduction is not a GEMM this kernel runs
+    if (G > MAX_G || m_capacity > 0x7fffffffLL || N > 0x7fffffffLL || K > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+    if (!group_offsets || !A || !sA || !B || !sB || !C) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(C) || (reinterpret_cast<uintptr_t>(sA) & 3) ||
+        (reinterpret_cast<uintptr_t>(sB) & 3) || (sC && (reinterpret_cast<uintptr_t>(sC) & 3)))
+        return MOE_ERR_INVALID_ARG;
+    int rc = prepare_kernel();
+    if (rc != MOE_OK) return rc;
+    auto enc = encode_fn();
+    if (!enc) return MOE_ERR_CUDA;
+
+    CUtensorMap tmA, tmB;
+    {
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(m_capacity)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+        cuuint32_t box[2] = {128, 128};
+        cuuint32_t es[2] = {1, 1};
+        if (enc(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(A), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MOE_ERR_CUDA;
+    }
+    {
+        cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(G)};
+        cuuint64_t strides[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N * K)};
+        cuuint32_t box[3] = {128, 128, 1};
+        cuuint32_t es[3] = {1, 1, 1};
+        if (enc(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(B), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MOE_ERR_CUDA;
+    }
+    const int grid = num_sms();
+    grouped_gemm_kernel<<<grid, THREADS, SMEM_BYTES, as_stream(stream)>>>(
+        tmA, tmB, group_offsets, G, m_capacity, static_cast<int>(N), static_cast<int>(K), sA, sB, epilogue, C,
+        sC, status);
+    return launch_status();
+}

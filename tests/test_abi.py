@@ -1,0 +1,80 @@
+"""The C-ABI library loads, exports every entry point the header declares, and
+rejects bad arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z][a-z0-9_]*)\s*\(", src)) - {"sizeof"})
+
+
+def test_header_parses_to_entry_points():
+    names = _declared()
+    for must in ["moe_route", "moe_permute", "fp8_quant_1x128", "fp8_grouped_gemm_blockscaled",
+                 "swiglu_requant", "moe_combine", "moe_bias_update"]:
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    from sparse_moe_layer_group_b200 import _abi
+    lib = ctypes.CDLL(_abi.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert set(_declared()) == set(_abi.EXPORTED)
+
+
+def test_status_strings_and_version():
+    from sparse_moe_layer_group_b200 import _abi
+    assert _abi.status_string(0) == "MOE_OK"
+    assert "INVALID_ARG" in _abi.status_string(1)
+    assert "unknown" in _abi.status_string(99)
+    assert _abi.abi_version() >= 1
+
+
+def test_workspace_size_scales_with_tokens():
+    from sparse_moe_layer_group_b200 import _abi
+    small = _abi.workspace_size(_abi.dims(64, 256, 16, 4, 4, 2, 128, 2.5))
+    big = _abi.workspace_size(_abi.dims(4096, 7168, 256, 8, 8, 4, 2048, 2.5))
+    assert big >= 4096 * 256 * 4 and small > 0 and small % 256 == 0
+
+
+def test_host_validation_rejects_before_launch():
+    from sparse_moe_layer_group_b200 import _abi as a
+    L = a._lib
+    # cols not a multiple of 128
+    assert L.fp8_quant_1x128(16, 4, 100, 16, 16, None, None) == a.MOE_ERR_INVALID_ARG
+    # NULL pointers
+    assert L.fp8_quant_1x128(None, 4, 128, None, None, None, None) == a.MOE_ERR_INVALID_ARG
+    # misaligned pointer
+    assert L.fp8_quant_1x128(18, 4, 128, 16, 16, None, None) == a.MOE_ERR_INVALID_ARG
+    # E not divisible by n_group; topk_group * group size < K; K too large
+    for d in [a.dims(8, 256, 16, 4, 3, 2, 128, 2.5), a.dims(8, 256, 16, 5, 4, 1, 128, 2.5),
+              a.dims(8, 256, 2048, 4, 4, 2, 128, 2.5)]:
+        rc = L.moe_route(ctypes.byref(d), 16, 16, 16, None, 16, 16, None, None, 0, None, None)
+        assert rc in (a.MOE_ERR_INVALID_ARG, a.MOE_ERR_UNSUPPORTED)
+    # workspace missing
+    d = a.dims(8, 256, 16, 4, 4, 2, 128, 2.5)
+    assert L.moe_route(ctypes.byref(d), 16, 16, 16, None, 16, 16, None, None, 0, None, None) == a.MOE_ERR_WORKSPACE
+    assert L.moe_permute(ctypes.byref(d), 16, None, None, 16, 16, 16, 16, None, None, 16, 8, None,
+                         None) == a.MOE_ERR_WORKSPACE
+    # GEMM: K not a multiple of 128, bad epilogue, SwiGLU without scale output
+    assert L.fp8_grouped_gemm_blockscaled(1, 16, 64, 256, 100, 16, 16, 16, 16, 0, 16, None, None,
+                                          None) == a.MOE_ERR_INVALID_ARG
+    assert L.fp8_grouped_gemm_blockscaled(1, 16, 64, 256, 128, 16, 16, 16, 16, 9, 16, None, None,
+                                          None) == a.MOE_ERR_INVALID_ARG
+    assert L.fp8_grouped_gemm_blockscaled(1, 16, 64, 256, 128, 16, 16, 16, 16, 2, 16, None, None,
+                                          None) == a.MOE_ERR_INVALID_ARG
+    # zero-size work is a no-op
+    assert L.fp8_grouped_gemm_blockscaled(0, 16, 64, 256, 128, 16, 16, 16, 16, 0, 16, None, None, None) == 0
+    assert L.fp8_quant_1x128(16, 0, 128, 16, 16, None, None) == 0
+    assert L.swiglu_requant(16, 4, 100, 16, 16, None, None) == a.MOE_ERR_INVALID_ARG
+    assert L.moe_bias_update(0, 4, 2, 0.001, 16, 16, None) == a.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(None, 16, 16, 16, None, 16, None, None) == a.MOE_ERR_INVALID_ARG
