@@ -215,6 +215,7 @@ def run_gpu(args, rank, world, local):
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
+        time.sleep(0.3)            # let the sampler start before the timed region
         t0.record(stream)
         for _ in range(args.steps):
             step(record=True)
@@ -355,14 +356,84 @@ def run_reference(args, rank, world):
     }
 
 
+# ----------------------------------------------------------------- single-kernel cases
+def run_case(args):
+    """One kernel alone on a profiling-sized case (a few GB on the device):
+    gemm1 = routed W13 GEMM with the SwiGLU+requant epilogue and gemm2 = routed
+    W2 GEMM, both on 64 experts x 128 rows at the DSV3 hidden/intermediate
+    sizes (1.9 GB / 0.9 GB of weights, larger than L2); router = moe_route at
+    T=4096, H=7168, E=256."""
+    import sparse_moe_layer_group_b200 as moe
+    abi = moe.abi
+    shape = synth.DSV3
+    H, I = shape.H, shape.I
+    E, rows = 64, 128
+    dev = "cuda"
+    ev = []
+    if args.case in ("gemm1", "gemm2"):
+        N, K = (2 * I, H) if args.case == "gemm1" else (H, I)
+        w = torch.empty(E, N, K, dtype=torch.uint8, device=dev)
+        sw = torch.empty(E, N // 128, K // 128, dtype=torch.float32, device=dev)
+        for e in range(E):
+            m = synth.expert_weight(N, K, shape.w_std, synth.seed_of(shape, synth.W13, e), device=dev)
+            abi.fp8_quant_128x128(m, w[e], sw[e])
+        a_bf = synth.activations(E * rows, K, 5, device=dev)
+        a = torch.empty(E * rows, K, dtype=torch.uint8, device=dev)
+        sa = torch.empty(E * rows, K // 128, dtype=torch.float32, device=dev)
+        abi.fp8_quant_1x128(a_bf, a, sa)
+        offs = torch.arange(0, E * rows + 1, rows, dtype=torch.int32, device=dev)
+        if args.case == "gemm1":
+            out = torch.empty(E * rows, N // 2, dtype=torch.uint8, device=dev)
+            so = torch.empty(E * rows, N // 256, dtype=torch.float32, device=dev)
+            run = lambda: abi.fp8_grouped_gemm_blockscaled(E, offs, E * rows, N, K, a, sa, w, sw,
+                                                          abi.MOE_EPI_SWIGLU_REQUANT, out, so)
+        else:
+            out = torch.empty(E * rows, N, dtype=torch.bfloat16, device=dev)
+            run = lambda: abi.fp8_grouped_gemm_blockscaled(E, offs, E * rows, N, K, a, sa, w, sw,
+                                                          abi.MOE_EPI_BF16, out)
+        nbytes = E * N * K + E * rows * K + E * rows * (N // 2 if args.case == "gemm1" else 2 * N)
+        flops = 2 * E * rows * N * K
+    elif args.case == "router":
+        T, E2 = shape.T, shape.E
+        x = synth.activations(T, H, 1, device=dev)
+        wr = synth.router_weights(E2, H, shape.wr_std, 2, device=dev)
+        b = torch.zeros(E2, dtype=torch.float32, device=dev)
+        d = abi.dims(T, H, E2, shape.K, shape.n_group, shape.topk_group, I, shape.rho)
+        idx = torch.empty(T, shape.K, dtype=torch.int32, device=dev)
+        wt = torch.empty(T, shape.K, dtype=torch.float32, device=dev)
+        sc = torch.empty(T, E2, dtype=torch.float32, device=dev)
+        run = lambda: abi.moe_route(d, x, wr, b, None, idx, wt, sc)
+        nbytes = T * H * 2 + E2 * H * 4 + T * E2 * 4
+        flops = 2 * T * E2 * H
+    else:
+        raise SystemExit(f"unknown case {args.case}")
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    for _ in range(args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run()
+        e1.record()
+        ev.append((e0, e1))
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    print(json.dumps({"case": args.case, "ms": round(ms, 4), "GB/s": round(nbytes / ms / 1e6, 1),
+                      "TFLOP/s": round(flops / ms / 1e9, 1), "algorithmic_bytes": nbytes, "flops": flops}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None, help="time one kernel alone: gemm1 | gemm2 | router")
     args = ap.parse_args()
+    if args.case:
+        run_case(args)
+        return
     rank, world, local = dist_setup(args.gpus)
     if args.impl == "reference":
         rec = run_reference(args, rank, world)

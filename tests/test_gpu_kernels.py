@@ -241,12 +241,16 @@ def test_combine(lib, T, H, E, K, shared):
     torch.cuda.synchronize()
     ref = oracle.combine(yperm.float().numpy(), row_of, w.numpy(),
                          ysh.float().numpy() if shared else None)
+    # fp32 accumulation error is bounded by the magnitudes summed, not the result
+    mag = oracle.combine(np.abs(yperm.float().numpy()), row_of, np.abs(w.numpy()),
+                         np.abs(ysh.float().numpy()) if shared else None)
     g32 = np_(out32)
-    assert np.all(np.abs(g32 - ref) <= 1e-5 * (np.abs(ref) + 1))
+    assert np.all(np.abs(g32 - ref) <= 4 * K * 2 ** -24 * mag)
     g16 = np_(out)
     r16 = oracle.round_bf16(ref)
-    assert np.all(np.abs(g16 - r16) <= bf16_ulp(r16))
-    assert normwise(g16, ref) < TOL_NORMWISE
+    # the bf16 store may flip at a rounding boundary: one bf16 step at most
+    assert np.all(np.abs(g16 - r16) <= bf16_ulp(r16) + 4 * K * 2 ** -24 * mag)
+    assert normwise(g16, r16) < TOL_NORMWISE
 
 
 # ---------------------------------------------------------------- bias update
