@@ -1,6 +1,8 @@
 """Build libmoe_b200.so (the C-ABI library) from csrc/*.cu for sm_100a.
 
-    python -m sparse_moe_layer_group_b200.build [--verbose-ptxas]
+    python sparse_moe_layer_group_b200/build.py [--verbose-ptxas]
+
+(run it by path: importing the package needs the library this script builds)
 
 Each .cu is compiled to an object in parallel, then linked into one shared
 library next to this file (in-tree, so it travels with the source tree).
