@@ -55,7 +55,8 @@ enum moe_status {
     MOE_ERR_INVALID_ARG = 1,
     MOE_ERR_UNSUPPORTED = 2,
     MOE_ERR_WORKSPACE = 3,
-    MOE_ERR_CUDA = 4
+    MOE_ERR_CUDA = 4,
+    MOE_ERR_TOO_LARGE = 5
 };
 
 /* Bits kernels OR into the optional device status word. */
@@ -143,6 +144,35 @@ int moe_route_select(const moe_dims *dims, const float *scores, const float *e_b
 int moe_permute(const moe_dims *dims, const int32_t *topk_idx, const uint8_t *xq, const float *xs,
                 int32_t *expert_load, int32_t *expert_offsets, int32_t *tok_of, int32_t *row_of,
                 uint8_t *aq, float *as, void *ws, size_t ws_bytes, int32_t *status, void *stream);
+
+/* moe_permute for callers that cannot allocate device memory.  The pages have
+ * no counterpart to this call; it exists for the host side.  Some callers may
+ * not call cudaMalloc at all: code that runs inside a host framework which owns
+ * every device buffer and forbids allocations in its kernels' call path, fixed
+ * memory budgets planned ahead of time (real-time or embedded deployments), and
+ * paths that must not synchronise the device, as cudaMalloc/cudaFree can.  This
+ * call takes no workspace: its scratch (the per-chunk expert counts) is a
+ * static device array of moe_permute_noalloc_max_scratch() bytes (1 MiB) that
+ * is part of the library's device image, so every GPU that loads the library
+ * holds it until the process exits.  The caller still passes every input and
+ * output, with the meaning, layout and limits of moe_permute.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture on the device.
+ *   - Problems whose counts exceed the scratch (ceil(T/128) * E * 4 bytes >
+ *     1 MiB, e.g. T > 131072 at E = 256) return MOE_ERR_TOO_LARGE.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     each call writes every count it reads before reading it, so nothing
+ *     needs clearing.  Calls whose work overlaps on the GPU (different
+ *     streams, or different host threads without ordering) race on the
+ *     array and give undefined results: order them on one stream.
+ *   - No cudaMalloc, cudaFree or allocating library routine is called.      */
+int moe_permute_noalloc(const moe_dims *dims, const int32_t *topk_idx, const uint8_t *xq, const float *xs,
+                        int32_t *expert_load, int32_t *expert_offsets, int32_t *tok_of, int32_t *row_of,
+                        uint8_t *aq, float *as, int32_t *status, void *stream);
+
+/* Size in bytes of moe_permute_noalloc's static scratch array. */
+size_t moe_permute_noalloc_max_scratch(void);
 
 /* Grouped FP8 GEMM with block scales, promoted every 128 of K
  * ([report-walkthrough] section 4.3; [infra-answer]: the tile/block scales

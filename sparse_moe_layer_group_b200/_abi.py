@@ -15,7 +15,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
-MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA = range(5)
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TOO_LARGE = range(6)
 MOE_FLAG_NONFINITE, MOE_FLAG_BAD_INDEX, MOE_FLAG_TIMEOUT, MOE_FLAG_BAD_OFFSETS = 1, 2, 4, 8
 MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_REQUANT = 0, 1, 2
 
@@ -35,7 +35,7 @@ class MoeDims(ctypes.Structure):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m sparse_moe_layer_group_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python sparse_moe_layer_group_b200/build.py` "
             "(there is no fallback path)")
     return ctypes.CDLL(LIB_PATH)
 
@@ -54,6 +54,8 @@ _SIGS = {
     "moe_route": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "moe_route_select": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P]),
     "moe_permute": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
+    "moe_permute_noalloc": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_permute_noalloc_max_scratch": (_SZ, []),
     "fp8_grouped_gemm_blockscaled": (ctypes.c_int, [_I32, _P, _I64, _I64, _I64, _P, _P, _P, _P, _I32,
                                                     _P, _P, _P, _P]),
     "swiglu_requant": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P]),
@@ -140,6 +142,18 @@ def moe_permute(d, topk_idx, xq, xs, expert_load, expert_offsets, tok_of, row_of
                                            _ptr(expert_load), _ptr(expert_offsets), _ptr(tok_of),
                                            _ptr(row_of), _ptr(aq), _ptr(as_), _ptr(ws), ws_bytes,
                                            _ptr(status), _stream(stream)))
+
+
+def moe_permute_noalloc(d, topk_idx, xq, xs, expert_load, expert_offsets, tok_of, row_of, aq, as_,
+                        status=None, stream=None):
+    """moe_permute without a workspace (static device scratch; see the header)."""
+    _check("moe_permute_noalloc", _lib.moe_permute_noalloc(
+        ctypes.byref(d), _ptr(topk_idx), _ptr(xq), _ptr(xs), _ptr(expert_load), _ptr(expert_offsets),
+        _ptr(tok_of), _ptr(row_of), _ptr(aq), _ptr(as_), _ptr(status), _stream(stream)))
+
+
+def moe_permute_noalloc_max_scratch() -> int:
+    return int(_lib.moe_permute_noalloc_max_scratch())
 
 
 def fp8_grouped_gemm_blockscaled(G, group_offsets, m_capacity, N, K, A, sA, B, sB, epilogue, C, sC=None,

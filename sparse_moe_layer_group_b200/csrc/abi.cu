@@ -13,6 +13,8 @@ MOE_API const char *moe_status_string(int status) {
         case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: valid arguments outside the kernels' limits";
         case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing or smaller than moe_workspace_size()";
         case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA runtime or launch error";
+        case MOE_ERR_TOO_LARGE:
+            return "MOE_ERR_TOO_LARGE: the problem needs more than the no-allocation call's static scratch";
         default: return "unknown moe_status";
     }
 }

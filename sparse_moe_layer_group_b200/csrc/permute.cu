@@ -165,3 +165,78 @@ MOE_API int moe_permute(const moe_dims *d, const int32_t *topk_idx, const uint8_
                                                 reinterpret_cast<uint4 *>(aq), as, d->H, d->K);
     return launch_status();
 }
+
+// ---------------------------------------------------------------------------
+// moe_permute_noalloc: the same permutation for callers that cannot allocate
+// device memory.  Its per-chunk expert counts live in the file-scope array
+// below instead of a caller workspace.  The array is a fixed part of every
+// device image of this library, so each GPU that loads the library holds its
+// 1 MiB until the process exits.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace moe {
+
+constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(1) << 20;   // 1 MiB: counts[n_chunks][E] int32
+constexpr int NOALLOC_MAX_DEVICES = 64;
+
+static __device__ __align__(256) int32_t g_perm_noalloc_scratch[NOALLOC_SCRATCH_BYTES / sizeof(int32_t)];
+
+// Device address of the scratch array, looked up once per device.  In host code
+// g_perm_noalloc_scratch names a host-side stand-in, not device memory, so the
+// kernels must be given the address cudaGetSymbolAddress returns.
+static int noalloc_scratch(int32_t **out) {
+    static std::mutex mu;
+    static int32_t *addr[NOALLOC_MAX_DEVICES] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NOALLOC_MAX_DEVICES) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_perm_noalloc_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+        addr[dev] = static_cast<int32_t *>(p);
+    }
+    *out = addr[dev];
+    return MOE_OK;
+}
+
+}  // namespace moe
+
+MOE_API size_t moe_permute_noalloc_max_scratch(void) { return moe::NOALLOC_SCRATCH_BYTES; }
+
+MOE_API int moe_permute_noalloc(const moe_dims *d, const int32_t *topk_idx, const uint8_t *xq, const float *xs,
+                                int32_t *expert_load, int32_t *expert_offsets, int32_t *tok_of,
+                                int32_t *row_of, uint8_t *aq, float *as, int32_t *status, void *stream) {
+    if (!d || d->T < 0 || d->E <= 0 || d->K <= 0 || d->H < 0) return MOE_ERR_INVALID_ARG;
+    if (d->E > PERM_MAX_E || d->K > 32) return MOE_ERR_UNSUPPORTED;
+    if (!expert_load || !expert_offsets) return MOE_ERR_INVALID_ARG;
+    const bool gather = xq || xs || aq || as;
+    if (gather && (!xq || !xs || !aq || !as || d->H % 128 != 0 || !aligned16(xq) || !aligned16(aq)))
+        return MOE_ERR_INVALID_ARG;
+    // the per-chunk counts must fit the static scratch
+    if (permute_workspace_bytes(d) > NOALLOC_SCRATCH_BYTES) return MOE_ERR_TOO_LARGE;
+    int32_t *counts = nullptr;
+    int rc = noalloc_scratch(&counts);
+    if (rc != MOE_OK) return rc;
+    cudaStream_t st = as_stream(stream);
+    if (d->T == 0) {
+        if (cudaMemsetAsync(expert_load, 0, sizeof(int32_t) * d->E, st) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (d->E + 1), st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    if (!topk_idx || !tok_of || !row_of) return MOE_ERR_INVALID_ARG;
+    // every count the later kernels read is written by perm_count_kernel first
+    // in this call, so the scratch needs no clearing between calls
+    const int n_chunks = (d->T + PERM_CHUNK - 1) / PERM_CHUNK;
+    const int thr = threads_for(d->E);
+    const size_t smem = static_cast<size_t>(PERM_CHUNK) * d->K * sizeof(int32_t);
+    perm_count_kernel<<<n_chunks, thr, smem, st>>>(topk_idx, counts, d->T, d->K, d->E, status);
+    perm_scan_kernel<<<1, thr, 0, st>>>(counts, n_chunks, d->E, expert_load, expert_offsets);
+    perm_place_kernel<<<n_chunks, thr, smem, st>>>(topk_idx, counts, expert_offsets, tok_of, row_of, d->T,
+                                                  d->K, d->E);
+    if (gather && d->H > 0)
+        perm_gather_kernel<<<d->T, 128, 0, st>>>(reinterpret_cast<const uint4 *>(xq), xs, row_of,
+                                                reinterpret_cast<uint4 *>(aq), as, d->H, d->K);
+    return launch_status();
+}
