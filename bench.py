@@ -402,7 +402,8 @@ def run_case(args):
         idx = torch.empty(T, shape.K, dtype=torch.int32, device=dev)
         wt = torch.empty(T, shape.K, dtype=torch.float32, device=dev)
         sc = torch.empty(T, E2, dtype=torch.float32, device=dev)
-        run = lambda: abi.moe_route(d, x, wr, b, None, idx, wt, sc)
+        ws = torch.empty(abi.workspace_size(d), dtype=torch.uint8, device=dev)
+        run = lambda: abi.moe_route(d, x, wr, b, None, idx, wt, sc, ws)
         nbytes = T * H * 2 + E2 * H * 4 + T * E2 * 4
         flops = 2 * T * E2 * H
     else:

@@ -10,95 +10,16 @@
 // keep_bf16 moe_gating); routed_scaling_factor multiplies the gates.
 //
 // Kernels:
-//   router_logits_kernel  SIMT fp32 GEMM x[T,H] (bf16) . W_r[E,H]^T, epilogue
-//                         adds the optional offset and applies the sigmoid.
-//   route_select_kernel   one warp per token: group scores, group pick, top-K,
+//   router_split_kernel / router_tc_kernel (router_tc.cu)  fp32-exact logits on
+//                         the tensor cores, split over K into partial sums.
+//   route_select_kernel   one warp per token: adds the partial logits in split
+//                         order, offset, sigmoid; group scores, group pick, top-K,
 //                         gates in float64 (exact sum of <= 32 fp32 values).
 #include <cfloat>
 
 #include "common.cuh"
 
 namespace moe {
-
-namespace rt {
-constexpr int BT = 64;      // tokens per CTA tile
-constexpr int BE = 64;      // experts per CTA tile
-constexpr int BK = 32;      // H chunk
-constexpr int THREADS = 256;
-}  // namespace rt
-
-// Each thread owns a 4 (tokens) x 4 (experts) block of the 64x64 tile.
-__global__ void __launch_bounds__(rt::THREADS) router_logits_kernel(
-    const __nv_bfloat16 *__restrict__ x, const float *__restrict__ w, const float *__restrict__ offset,
-    float *__restrict__ s_out, int T, int H, int E) {
-    __shared__ float xs[rt::BK][rt::BT + 4];
-    __shared__ float ws[rt::BK][rt::BE + 4];
-    const int tid = threadIdx.x;
-    const int t0 = blockIdx.x * rt::BT, e0 = blockIdx.y * rt::BE;
-    const int tr = tid / 16, tc = tid % 16;     // 16 x 16 threads
-    float acc[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
-
-    // load mapping: x tile 64 tokens x 32 h = 256 x (8 bf16); w tile 64 x 32 fp32 = 256 x 8 fp32
-    const int lrow = tid / 4, lcol = (tid % 4) * 8;
-    for (int k0 = 0; k0 < H; k0 += rt::BK) {
-        {
-            const int t = t0 + lrow;
-            float v[8];
-            if (t < T) {
-                const uint4 u = __ldg(reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(t) * H + k0 + lcol));
-                v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
-                v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z); v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) xs[lcol + i][lrow] = v[i];
-        }
-        {
-            const int e = e0 + lrow;
-            float4 a = make_float4(0, 0, 0, 0), b = make_float4(0, 0, 0, 0);
-            if (e < E) {
-                const float4 *p = reinterpret_cast<const float4 *>(w + static_cast<int64_t>(e) * H + k0 + lcol);
-                a = __ldg(p);
-                b = __ldg(p + 1);
-            }
-            ws[lcol + 0][lrow] = a.x; ws[lcol + 1][lrow] = a.y; ws[lcol + 2][lrow] = a.z; ws[lcol + 3][lrow] = a.w;
-            ws[lcol + 4][lrow] = b.x; ws[lcol + 5][lrow] = b.y; ws[lcol + 6][lrow] = b.z; ws[lcol + 7][lrow] = b.w;
-        }
-        __syncthreads();
-#pragma unroll 8
-        for (int k = 0; k < rt::BK; ++k) {
-            float xa[4], wb[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) xa[i] = xs[k][tr + 16 * i];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) wb[j] = ws[k][tc + 16 * j];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xa[i], wb[j], acc[i][j]);
-        }
-        __syncthreads();
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int t = t0 + tr + 16 * i;
-        if (t >= T) continue;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int e = e0 + tc + 16 * j;
-            if (e >= E) continue;
-            float l = acc[i][j];
-            if (offset) l = __fadd_rn(l, __ldg(offset + e));
-            s_out[static_cast<int64_t>(t) * E + e] = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l)));
-        }
-    }
-}
 
 // (value, index) order used for every ranking: larger value first, then the
 // lower index.
@@ -118,38 +39,54 @@ __device__ __forceinline__ void warp_best(float &v, int &i) {
 constexpr int SEL_WARPS = 8;
 constexpr int SEL_MAX_E = 1024;
 
-// One warp per token.  Per-warp shared row of r = s + b.
+// One warp per token.  The affinities come either given (s_in [T, E]) or as
+// n_split fp32 partial logits [n_split, T, E] from the tensor-core router, which
+// are added in split order (a fixed order, so results are deterministic), offset
+// and passed through the sigmoid here.  r = s + b is formed where it is used.
 __global__ void __launch_bounds__(SEL_WARPS * 32) route_select_kernel(
-    const float *__restrict__ s, const float *__restrict__ bias, int32_t *__restrict__ topk_idx,
-    float *__restrict__ topk_w, int T, int E, int K, int n_group, int topk_group, float rho) {
-    extern __shared__ float sh[];   // SEL_WARPS * E floats
+    const float *__restrict__ s_in, const float *__restrict__ partial, int n_split,
+    const float *__restrict__ offset, float *__restrict__ s_out, const float *__restrict__ bias,
+    int32_t *__restrict__ topk_idx, float *__restrict__ topk_w, int T, int E, int K, int n_group,
+    int topk_group, float rho) {
+    extern __shared__ float sh[];   // SEL_WARPS * E affinities
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int t = blockIdx.x * SEL_WARPS + wid;
     if (t >= T) return;
-    float *r = sh + wid * E;
-    const float *srow = s + static_cast<int64_t>(t) * E;
-    for (int e = lane; e < E; e += 32) r[e] = __fadd_rn(srow[e], __ldg(bias + e));
+    float *srow = sh + wid * E;
+    if (partial) {
+        const int64_t plane = static_cast<int64_t>(T) * E;
+        for (int e = lane; e < E; e += 32) {
+            const float *p = partial + static_cast<int64_t>(t) * E + e;
+            float l = p[0];
+            for (int q = 1; q < n_split; ++q) l = __fadd_rn(l, p[q * plane]);
+            if (offset) l = __fadd_rn(l, __ldg(offset + e));
+            const float sv = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l)));
+            srow[e] = sv;
+            if (s_out) s_out[static_cast<int64_t>(t) * E + e] = sv;
+        }
+    } else {
+        for (int e = lane; e < E; e += 32) srow[e] = s_in[static_cast<int64_t>(t) * E + e];
+    }
     __syncwarp();
     const int gs = E / n_group;
-    // group scores: lane g scans its group for the two largest values
+    // group scores: lane g scans its group for the two largest values of r
     float gscore = -FLT_MAX;
-    bool gvalid = false;
-    if (lane < n_group) {
+    const bool gvalid = lane < n_group;
+    if (gvalid) {
         float m1 = -FLT_MAX, m2 = -FLT_MAX;
         for (int j = 0; j < gs; ++j) {
-            const float v = r[lane * gs + j];
+            const int e = lane * gs + j;
+            const float v = __fadd_rn(srow[e], __ldg(bias + e));
             if (v > m1) { m2 = m1; m1 = v; } else if (v > m2) { m2 = v; }
         }
         gscore = gs == 1 ? m1 : __fadd_rn(m1, m2);
-        gvalid = true;
     }
     // keep the topk_group best groups (ties to the lower group)
     uint32_t kept = 0;
     bool taken_g = !gvalid;
     for (int round = 0; round < topk_group; ++round) {
-        float v = taken_g ? -FLT_MAX : gscore;
+        float v = taken_g ? -INFINITY : gscore;
         int i = taken_g ? 0x7fffffff : lane;
-        if (taken_g) v = -INFINITY;
         warp_best(v, i);
         kept |= 1u << i;
         if (lane == i) taken_g = true;
@@ -165,7 +102,7 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) route_select_kernel(
         for (int j = 0; j < per_lane; ++j) {
             const int e = lane + 32 * j;
             if (e >= E || (taken >> j & 1u) || !(kept >> (e / gs) & 1u)) continue;
-            const float v = r[e];
+            const float v = __fadd_rn(srow[e], __ldg(bias + e));
             if (better(v, e, bv, bi)) { bv = v; bi = e; }
         }
         warp_best(bv, bi);
@@ -193,19 +130,25 @@ static int check_route_dims(const moe_dims *d) {
     return MOE_OK;
 }
 
-static int launch_select(const moe_dims *d, const float *scores, const float *e_bias, int32_t *idx,
-                         float *w, cudaStream_t st) {
+static int launch_select(const moe_dims *d, const float *s_in, const float *partial, int n_split,
+                         const float *offset, float *s_out, const float *e_bias, int32_t *idx, float *w,
+                         cudaStream_t st) {
     const int blocks = (d->T + SEL_WARPS - 1) / SEL_WARPS;
     const size_t smem = static_cast<size_t>(SEL_WARPS) * d->E * sizeof(float);
-    route_select_kernel<<<blocks, SEL_WARPS * 32, smem, st>>>(scores, e_bias, idx, w, d->T, d->E, d->K,
-                                                              d->n_group, d->topk_group,
+    route_select_kernel<<<blocks, SEL_WARPS * 32, smem, st>>>(s_in, partial, n_split, offset, s_out, e_bias, idx,
+                                                              w, d->T, d->E, d->K, d->n_group, d->topk_group,
                                                               d->routed_scaling_factor);
     return launch_status();
 }
 
+int router_splits(int T, int E, int H);
+size_t router_tc_ws_bytes(int T, int E, int H);
+int launch_router_tc(const void *x, const float *w, int T, int E, int H, void *ws, float **partial_out,
+                     int *n_split_out, int32_t *status, cudaStream_t st);
+
 size_t route_workspace_bytes(const moe_dims *d) {
-    // the [T, E] fp32 affinities when the caller does not want them
-    return (static_cast<size_t>(d->T) * d->E * sizeof(float) + 255) & ~static_cast<size_t>(255);
+    // three bf16 pieces of W_r and the split-K partial logits
+    return router_tc_ws_bytes(d->T, d->E, d->H);
 }
 
 }  // namespace moe
@@ -215,24 +158,18 @@ using namespace moe;
 MOE_API int moe_route(const moe_dims *d, const void *x, const float *w_router, const float *e_bias,
                       const float *router_offset, int32_t *topk_idx, float *topk_w, float *scores,
                       void *ws, size_t ws_bytes, int32_t *status, void *stream) {
-    (void)status;
     int rc = check_route_dims(d);
     if (rc != MOE_OK) return rc;
     if (d->T == 0) return MOE_OK;
     if (!x || !w_router || !e_bias || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
-    float *s = scores;
-    if (!s) {
-        if (!ws || ws_bytes < route_workspace_bytes(d)) return MOE_ERR_WORKSPACE;
-        s = reinterpret_cast<float *>(ws);
-    }
+    if (!ws || ws_bytes < route_workspace_bytes(d) || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOE_ERR_WORKSPACE;
     cudaStream_t st = as_stream(stream);
-    dim3 grid((d->T + rt::BT - 1) / rt::BT, (d->E + rt::BE - 1) / rt::BE);
-    router_logits_kernel<<<grid, rt::THREADS, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), w_router,
-                                                       router_offset, s, d->T, d->H, d->E);
-    rc = launch_status();
+    float *partial = nullptr;
+    int n_split = 0;
+    rc = launch_router_tc(x, w_router, d->T, d->E, d->H, ws, &partial, &n_split, status, st);
     if (rc != MOE_OK) return rc;
-    return launch_select(d, s, e_bias, topk_idx, topk_w, st);
+    return launch_select(d, nullptr, partial, n_split, router_offset, scores, e_bias, topk_idx, topk_w, st);
 }
 
 MOE_API int moe_route_select(const moe_dims *d, const float *scores, const float *e_bias,
@@ -241,5 +178,5 @@ MOE_API int moe_route_select(const moe_dims *d, const float *scores, const float
     if (rc != MOE_OK) return rc;
     if (d->T == 0) return MOE_OK;
     if (!scores || !e_bias || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
-    return launch_select(d, scores, e_bias, topk_idx, topk_w, as_stream(stream));
+    return launch_select(d, scores, nullptr, 0, nullptr, nullptr, e_bias, topk_idx, topk_w, as_stream(stream));
 }

@@ -98,7 +98,8 @@ def test_router_scores_close_to_float64(lib, shape):
     idx = torch.empty(T, shape.K, dtype=torch.int32, device="cuda")
     w = torch.empty(T, shape.K, dtype=torch.float32, device="cuda")
     sc = torch.empty(T, E, dtype=torch.float32, device="cuda")
-    lib.moe_route(d, cuda(x), cuda(wr), cuda(b), cuda(off), idx, w, sc)
+    ws = torch.empty(lib.workspace_size(d), dtype=torch.uint8, device="cuda")
+    lib.moe_route(d, cuda(x), cuda(wr), cuda(b), cuda(off), idx, w, sc, ws)
     torch.cuda.synchronize()
     ref = oracle.router_scores(x.float().numpy(), wr.numpy(), off.numpy())
     assert np.max(np.abs(np_(sc) - ref) / ref) < 1e-5
