@@ -156,12 +156,13 @@ def build_layer(shape: synth.MoEShape, T: int):
 
 
 def gemm1_bytes(layer, touched: int) -> int:
-    """Algorithmic HBM bytes of the routed GEMM1 launch (W13 of the touched
-    experts + permuted A codes/scales + requantised output codes/scales)."""
+    """Algorithmic HBM bytes of the W13 grouped GEMM launch: W13 of the touched
+    routed experts and of the shared expert, the T*K + T A rows (codes +
+    scales) and the requantised output rows (codes + scales)."""
     T, H, K, I = layer.T, layer.H, layer.K, layer.I
-    w = touched * (2 * I * H + (2 * I // 128) * (H // 128) * 4)
-    a = T * K * (H + (H // 128) * 4)
-    o = T * K * (I + (I // 128) * 4)
+    w = (touched + 1) * (2 * I * H + (2 * I // 128) * (H // 128) * 4)
+    a = (T * K + T) * (H + (H // 128) * 4)
+    o = (T * K + T) * (I + (I // 128) * 4)
     return w + a + o
 
 
@@ -180,31 +181,11 @@ def run_gpu(args, rank, world, local):
     g1_events = []
 
     def step(record=False):
-        abi = moe.abi
-        st = layer.status
-        abi.moe_route(layer.d, x, layer.w_router, layer.e_bias, None, layer.topk_idx, layer.topk_w, layer.scores,
-                      layer.ws, st)
-        abi.fp8_quant_1x128(x, layer.xq, layer.xs, st)
-        abi.moe_permute(layer.d, layer.topk_idx, layer.xq, layer.xs, layer.load, layer.offsets, layer.tok_of,
-                        layer.row_of, layer.aq, layer.as_, layer.ws, st)
-        qw = layer.qw
+        ev = None
         if record:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-        abi.fp8_grouped_gemm_blockscaled(layer.E, layer.offsets, T * layer.K, 2 * layer.I, layer.H, layer.aq,
-                                         layer.as_, qw.w13, qw.s13, abi.MOE_EPI_SWIGLU_REQUANT, layer.actq,
-                                         layer.acts, st)
-        if record:
-            e1.record(stream)
-            g1_events.append((e0, e1))
-        abi.fp8_grouped_gemm_blockscaled(layer.E, layer.offsets, T * layer.K, layer.H, layer.I, layer.actq,
-                                         layer.acts, qw.w2, qw.s2, abi.MOE_EPI_BF16, layer.yperm, None, st)
-        abi.fp8_grouped_gemm_blockscaled(1, layer.sh_offsets, T, 2 * layer.I, layer.H, layer.xq, layer.xs,
-                                         qw.sh13, qw.sh13s, abi.MOE_EPI_SWIGLU_REQUANT, layer.sh_actq,
-                                         layer.sh_acts, st)
-        abi.fp8_grouped_gemm_blockscaled(1, layer.sh_offsets, T, layer.H, layer.I, layer.sh_actq, layer.sh_acts,
-                                         qw.sh2, qw.sh2s, abi.MOE_EPI_BF16, layer.ysh, None, st)
-        abi.moe_combine(layer.d, layer.yperm, layer.row_of, layer.topk_w, layer.ysh, layer.out, None)
+            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            g1_events.append(ev)
+        layer.forward(x, gemm1_events=ev)
         layer.bias_update(gamma)
 
     launches_per_step = moe.LAUNCHES_PER_FORWARD + 1
@@ -261,7 +242,7 @@ def run_gpu(args, rank, world, local):
     fp8_peak = 2.0 * pk["bf16_tflops"]          # nominal fp8:bf16 ratio 2 on the measured bf16 burst
     g1_bytes = gemm1_bytes(layer, touched)
     g1_gbs = g1_bytes / (g1_ms / 1e3) / 1e9
-    g1_tflops = 2 * T * layer.K * 2 * layer.I * layer.H / (g1_ms / 1e3) / 1e12
+    g1_tflops = 2 * (T * layer.K + T) * 2 * layer.I * layer.H / (g1_ms / 1e3) / 1e12
     rec = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -281,7 +262,7 @@ def run_gpu(args, rank, world, local):
         "gemm_tflops": round(gemm_flops_step / (ms_max / args.steps / 1e3) / 1e12, 1),
         "gemm_pct_fp8_peak": round(100 * gemm_flops_step / (ms_max / args.steps / 1e3) / 1e12 / fp8_peak, 1),
         "roofline": {
-            "kernel": "grouped_gemm_kernel (routed W13, SwiGLU+requant epilogue)",
+            "kernel": "grouped_gemm_kernel (W13 of 256 routed + 1 shared expert, SwiGLU+requant epilogue)",
             "bound": "hbm", "achieved": round(g1_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(g1_gbs / pk["hbm_gbs"], 3), "traffic": None, "peak_kind": pk_kind,
             "launch_ms": round(g1_ms, 4), "algorithmic_bytes": g1_bytes, "touched_experts": touched,

@@ -3,18 +3,23 @@
 PyTorch only allocates device memory and supplies the stream; every step of
 the forward runs in the library's kernels:
 
-  1  moe_route        router GEMM + sigmoid, group-limited top-K, gates
-  2  fp8_quant_1x128  x -> e4m3 codes + 1x128 scales
+  1  moe_route        router GEMM (tensor cores) + sigmoid, group-limited top-K,
+                      gates (3 kernels)
+  2  fp8_quant_1x128  x -> e4m3 codes + 1x128 scales, written straight into the
+                      last T rows of the expert-ordered A matrix
   3  moe_permute      stable counting sort by expert + row gather (4 kernels)
-  4  grouped GEMM     routed experts' W13, SwiGLU + 1x128 requant epilogue
-  5  grouped GEMM     routed experts' W2 -> bf16 rows
-  6  grouped GEMM     shared expert W13 (one group over all T rows), SwiGLU
-  7  grouped GEMM     shared expert W2 -> bf16
-  8  moe_combine      gate-weighted sum of the K rows + shared row -> bf16
-  (9 moe_bias_update  after the step, from the expert loads of step 3)
+                      into the first T*K rows
+  4  grouped GEMM     W13 of the E routed experts and, as group E, of the
+                      shared expert over the T token rows; SwiGLU + 1x128
+                      requant fused
+  5  grouped GEMM     W2 of the same E + 1 groups -> bf16 rows
+  6  moe_combine      gate-weighted sum of the K rows + the shared row -> bf16
+  (7 moe_bias_update  after the step, from the expert loads of step 3)
 
-Order and arithmetic follow the "DeepSeek-V3 technical report" walkthrough
-(2kiu.com), sections 3.2, 3.4 and 4.3.
+Treating the shared expert as one more group of the same two launches lets its
+compute-bound tiles run in the tail of the weight-bound routed tiles.  Order and
+arithmetic follow the "DeepSeek-V3 technical report" walkthrough (2kiu.com),
+sections 3.2, 3.4 and 4.3.
 """
 from __future__ import annotations
 
@@ -25,58 +30,51 @@ import torch
 
 from . import _abi as abi
 
-LAUNCHES_PER_FORWARD = 12   # 2 route + 1 quant + 4 permute + 4 GEMM + 1 combine
+LAUNCHES_PER_FORWARD = 11   # 3 route + 1 quant + 4 permute + 2 GEMM + 1 combine
 
 
 @dataclass
 class QuantWeights:
-    """128x128 block-quantised expert weights resident in HBM.
+    """128x128 block-quantised expert weights resident in HBM, routed experts
+    0..E-1 and the shared expert as expert E.
 
-    w13 e4m3 [E, 2I, H] (gate rows 0..I-1, up rows I..2I-1), s13 fp32
-    [E, 2I/128, H/128]; w2 e4m3 [E, H, I], s2 fp32 [E, H/128, I/128];
-    sh13/sh13s and sh2/sh2s the same for the shared expert with E = 1."""
+    w13 e4m3 [E+1, 2I, H] (gate rows 0..I-1, up rows I..2I-1), s13 fp32
+    [E+1, 2I/128, H/128]; w2 e4m3 [E+1, H, I], s2 fp32 [E+1, H/128, I/128]."""
     w13: torch.Tensor
     s13: torch.Tensor
     w2: torch.Tensor
     s2: torch.Tensor
-    sh13: torch.Tensor
-    sh13s: torch.Tensor
-    sh2: torch.Tensor
-    sh2s: torch.Tensor
+
+    @property
+    def E(self) -> int:
+        return self.w13.shape[0] - 1
 
     @property
     def nbytes(self) -> int:
-        return sum(t.numel() * t.element_size() for t in
-                   (self.w13, self.s13, self.w2, self.s2, self.sh13, self.sh13s, self.sh2, self.sh2s))
+        return sum(t.numel() * t.element_size() for t in (self.w13, self.s13, self.w2, self.s2))
 
     @staticmethod
     def from_master(master: Callable[[str, int], torch.Tensor], E: int, H: int, I: int,
                     device="cuda", status: Optional[torch.Tensor] = None) -> "QuantWeights":
         """Quantise master weights expert by expert with fp8_quant_128x128.
 
-        master(kind, e) returns a bf16 device tensor: kind "w13" -> [2I, H],
-        "w2" -> [H, I]; e = -1 is the shared expert."""
+        master(kind, e) returns a bf16 tensor: kind "w13" -> [2I, H], "w2" ->
+        [H, I]; e = -1 is the shared expert (stored as expert E)."""
         u8 = dict(dtype=torch.uint8, device=device)
         f32 = dict(dtype=torch.float32, device=device)
-        w13 = torch.empty(E, 2 * I, H, **u8)
-        s13 = torch.empty(E, 2 * I // 128, H // 128, **f32)
-        w2 = torch.empty(E, H, I, **u8)
-        s2 = torch.empty(E, H // 128, I // 128, **f32)
-        sh13 = torch.empty(1, 2 * I, H, **u8)
-        sh13s = torch.empty(1, 2 * I // 128, H // 128, **f32)
-        sh2 = torch.empty(1, H, I, **u8)
-        sh2s = torch.empty(1, H // 128, I // 128, **f32)
+        w13 = torch.empty(E + 1, 2 * I, H, **u8)
+        s13 = torch.empty(E + 1, 2 * I // 128, H // 128, **f32)
+        w2 = torch.empty(E + 1, H, I, **u8)
+        s2 = torch.empty(E + 1, H // 128, I // 128, **f32)
         for e in range(-1, E):
+            slot = E if e < 0 else e
             a = master("w13", e).to(device).contiguous()
+            abi.fp8_quant_128x128(a, w13[slot], s13[slot], status)
+            del a
             b = master("w2", e).to(device).contiguous()
-            if e < 0:
-                abi.fp8_quant_128x128(a, sh13[0], sh13s[0], status)
-                abi.fp8_quant_128x128(b, sh2[0], sh2s[0], status)
-            else:
-                abi.fp8_quant_128x128(a, w13[e], s13[e], status)
-                abi.fp8_quant_128x128(b, w2[e], s2[e], status)
-            del a, b
-        return QuantWeights(w13, s13, w2, s2, sh13, sh13s, sh2, sh2s)
+            abi.fp8_quant_128x128(b, w2[slot], s2[slot], status)
+            del b
+        return QuantWeights(w13, s13, w2, s2)
 
 
 class MoELayer:
@@ -90,6 +88,7 @@ class MoELayer:
         self.d = abi.dims(T, H, E, K, n_group, topk_group, I, rho)
         self.w_router, self.e_bias, self.router_offset = w_router, e_bias, router_offset
         self.qw = weights
+        assert weights.E == E, "weights hold E routed experts plus the shared one"
         dev = dict(device=device)
         i32 = dict(dtype=torch.int32, **dev)
         f32 = dict(dtype=torch.float32, **dev)
@@ -101,47 +100,53 @@ class MoELayer:
         self.scores = torch.empty(T, E, **f32)
         ws_bytes = max(abi.workspace_size(self.d), 256)
         self.ws = torch.empty((ws_bytes + 255) // 256 * 256, **u8)
-        self.xq = torch.empty(T, H, **u8)
-        self.xs = torch.empty(T, H // 128, **f32)
+        # A of both GEMM launches: rows 0..T*K-1 the routed (token, slot) pairs
+        # in expert order, rows T*K..T*K+T-1 the tokens themselves (shared expert)
+        self.aq = torch.empty(TK + T, H, **u8)
+        self.as_ = torch.empty(TK + T, H // 128, **f32)
+        self.xq = self.aq[TK:]
+        self.xs = self.as_[TK:]
         self.load = torch.empty(E, **i32)
-        self.offsets = torch.empty(E + 1, **i32)
+        # group offsets of the E + 1 groups: moe_permute writes entries 0..E,
+        # entry E + 1 closes the shared group
+        self.offsets_all = torch.full((E + 2,), TK + T, **i32)
+        self.offsets = self.offsets_all[:E + 1]
         self.tok_of = torch.empty(TK, **i32)
         self.row_of = torch.empty(TK, **i32)
-        self.aq = torch.empty(TK, H, **u8)
-        self.as_ = torch.empty(TK, H // 128, **f32)
-        self.actq = torch.empty(TK, I, **u8)
-        self.acts = torch.empty(TK, I // 128, **f32)
-        self.yperm = torch.empty(TK, H, **bf)
-        self.sh_actq = torch.empty(T, I, **u8)
-        self.sh_acts = torch.empty(T, I // 128, **f32)
-        self.ysh = torch.empty(T, H, **bf)
+        self.actq = torch.empty(TK + T, I, **u8)
+        self.acts = torch.empty(TK + T, I // 128, **f32)
+        self.yperm = torch.empty(TK + T, H, **bf)
+        self.ysh = self.yperm[TK:]
         self.out = torch.empty(T, H, **bf)
         self.out_f32 = None
         self.status = torch.zeros(1, **i32)
-        self.sh_offsets = torch.tensor([0, T], **i32)
 
-    def forward(self, x: torch.Tensor, out_f32: bool = False, stream=None) -> torch.Tensor:
-        """x bf16 [T, H] on the device -> out bf16 [T, H] (self.out)."""
+    def forward(self, x: torch.Tensor, out_f32: bool = False, stream=None, gemm1_events=None) -> torch.Tensor:
+        """x bf16 [T, H] on the device -> out bf16 [T, H] (self.out).
+
+        gemm1_events, if given, is a (start, end) pair of CUDA events recorded
+        around the W13 grouped GEMM on the launching stream."""
         T, H, E, K, I = self.T, self.H, self.E, self.K, self.I
         if T == 0:
             return self.out
         if out_f32 and self.out_f32 is None:
             self.out_f32 = torch.empty(T, H, dtype=torch.float32, device=self.out.device)
         st = self.status
+        M = T * K + T
         abi.moe_route(self.d, x, self.w_router, self.e_bias, self.router_offset, self.topk_idx,
                       self.topk_w, self.scores, self.ws, st, stream)
         abi.fp8_quant_1x128(x, self.xq, self.xs, st, stream)
         abi.moe_permute(self.d, self.topk_idx, self.xq, self.xs, self.load, self.offsets, self.tok_of,
                         self.row_of, self.aq, self.as_, self.ws, st, stream)
         qw = self.qw
-        abi.fp8_grouped_gemm_blockscaled(E, self.offsets, T * K, 2 * I, H, self.aq, self.as_, qw.w13, qw.s13,
+        if gemm1_events is not None:
+            gemm1_events[0].record(torch.cuda.current_stream() if stream is None else stream)
+        abi.fp8_grouped_gemm_blockscaled(E + 1, self.offsets_all, M, 2 * I, H, self.aq, self.as_, qw.w13, qw.s13,
                                          abi.MOE_EPI_SWIGLU_REQUANT, self.actq, self.acts, st, stream)
-        abi.fp8_grouped_gemm_blockscaled(E, self.offsets, T * K, H, I, self.actq, self.acts, qw.w2, qw.s2,
+        if gemm1_events is not None:
+            gemm1_events[1].record(torch.cuda.current_stream() if stream is None else stream)
+        abi.fp8_grouped_gemm_blockscaled(E + 1, self.offsets_all, M, H, I, self.actq, self.acts, qw.w2, qw.s2,
                                          abi.MOE_EPI_BF16, self.yperm, None, st, stream)
-        abi.fp8_grouped_gemm_blockscaled(1, self.sh_offsets, T, 2 * I, H, self.xq, self.xs, qw.sh13, qw.sh13s,
-                                         abi.MOE_EPI_SWIGLU_REQUANT, self.sh_actq, self.sh_acts, st, stream)
-        abi.fp8_grouped_gemm_blockscaled(1, self.sh_offsets, T, H, I, self.sh_actq, self.sh_acts, qw.sh2,
-                                         qw.sh2s, abi.MOE_EPI_BF16, self.ysh, None, st, stream)
         abi.moe_combine(self.d, self.yperm, self.row_of, self.topk_w, self.ysh, self.out,
                         self.out_f32 if out_f32 else None, stream)
         return self.out
