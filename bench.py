@@ -5,7 +5,8 @@
 
 A step is one pass of the whole hot path over one batch: router + top-K,
 1x128 quantisation, permutation, routed grouped GEMMs (SwiGLU + requant fused),
-shared expert, combine, and the per-batch expert-bias update.  Inputs are
+shared expert, combine, and the per-batch expert-bias update (written to a
+separate buffer, so every step routes with the configured bias b = 0).  Inputs are
 synthetic (seeded) with the DeepSeek-V3 layer shape: T=4096 tokens, hidden 7168,
 256 routed + 1 shared expert, top-8 with 8 groups / 4 kept, expert intermediate
 2048, routed_scaling_factor 2.5; all 257 experts' E4M3 weights (11.3 GB) are
@@ -179,6 +180,7 @@ def run_gpu(args, rank, world, local):
 
     # the dominant kernel's launches are bracketed with events on the same stream
     g1_events = []
+    b_next = layer.e_bias.clone()
 
     def step(record=False):
         ev = None
@@ -186,7 +188,9 @@ def run_gpu(args, rank, world, local):
             ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             g1_events.append(ev)
         layer.forward(x, gemm1_events=ev)
-        layer.bias_update(gamma)
+        # the bias update runs every step; its result goes to b_next so the
+        # workload keeps the configured routing bias b = 0
+        layer.bias_update(gamma, bias=b_next)
 
     launches_per_step = moe.LAUNCHES_PER_FORWARD + 1
     for _ in range(args.warmup):
@@ -227,7 +231,7 @@ def run_gpu(args, rank, world, local):
     for _ in range(args.steps):
         xd.copy_(xh, non_blocking=True)
         layer.forward(xd)
-        layer.bias_update(gamma)
+        layer.bias_update(gamma, bias=b_next)
         outh.copy_(layer.out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -351,29 +355,40 @@ def run_case(args):
     E, rows = 64, 128
     dev = "cuda"
     ev = []
-    if args.case in ("gemm1", "gemm2"):
-        N, K = (2 * I, H) if args.case == "gemm1" else (H, I)
+    if args.case in ("gemm1", "gemm2", "gemm1_x256", "gemm1_skew"):
+        N, K = (H, I) if args.case == "gemm2" else (2 * I, H)
         w = torch.empty(E, N, K, dtype=torch.uint8, device=dev)
         sw = torch.empty(E, N // 128, K // 128, dtype=torch.float32, device=dev)
         for e in range(E):
             m = synth.expert_weight(N, K, shape.w_std, synth.seed_of(shape, synth.W13, e), device=dev)
             abi.fp8_quant_128x128(m, w[e], sw[e])
-        a_bf = synth.activations(E * rows, K, 5, device=dev)
-        a = torch.empty(E * rows, K, dtype=torch.uint8, device=dev)
-        sa = torch.empty(E * rows, K // 128, dtype=torch.float32, device=dev)
-        abi.fp8_quant_1x128(a_bf, a, sa)
-        offs = torch.arange(0, E * rows + 1, rows, dtype=torch.int32, device=dev)
-        if args.case == "gemm1":
-            out = torch.empty(E * rows, N // 2, dtype=torch.uint8, device=dev)
-            so = torch.empty(E * rows, N // 256, dtype=torch.float32, device=dev)
-            run = lambda: abi.fp8_grouped_gemm_blockscaled(E, offs, E * rows, N, K, a, sa, w, sw,
-                                                          abi.MOE_EPI_SWIGLU_REQUANT, out, so)
+        if args.case == "gemm1_x256":
+            sizes = [2 * rows] * E
+        elif args.case == "gemm1_skew":
+            # log-normal expert loads with mean 128 rows (spread like an unbalanced router)
+            g = synth.gen(11, "cpu")
+            wts = torch.exp(0.6 * torch.randn(E, generator=g, dtype=torch.float64))
+            sizes = torch.floor(wts / wts.sum() * E * rows).to(torch.int64).tolist()
         else:
-            out = torch.empty(E * rows, N, dtype=torch.bfloat16, device=dev)
-            run = lambda: abi.fp8_grouped_gemm_blockscaled(E, offs, E * rows, N, K, a, sa, w, sw,
-                                                          abi.MOE_EPI_BF16, out)
-        nbytes = E * N * K + E * rows * K + E * rows * (N // 2 if args.case == "gemm1" else 2 * N)
-        flops = 2 * E * rows * N * K
+            sizes = [rows] * E
+        Mrows = int(sum(sizes))
+        a_bf = synth.activations(Mrows, K, 5, device=dev)
+        a = torch.empty(Mrows, K, dtype=torch.uint8, device=dev)
+        sa = torch.empty(Mrows, K // 128, dtype=torch.float32, device=dev)
+        abi.fp8_quant_1x128(a_bf, a, sa)
+        offs = torch.tensor([0] + list(np.cumsum(sizes)), dtype=torch.int32, device=dev)
+        mode = {"auto": 0, "single": abi.MOE_GEMM_SINGLE_CTA, "pair": abi.MOE_GEMM_PAIR_CTA}[args.gemm_mode]
+        if args.case != "gemm2":
+            out = torch.empty(Mrows, N // 2, dtype=torch.uint8, device=dev)
+            so = torch.empty(Mrows, N // 256, dtype=torch.float32, device=dev)
+            run = lambda: abi.fp8_grouped_gemm_blockscaled(E, offs, Mrows, N, K, a, sa, w, sw,
+                                                          abi.MOE_EPI_SWIGLU_REQUANT | mode, out, so)
+        else:
+            out = torch.empty(Mrows, N, dtype=torch.bfloat16, device=dev)
+            run = lambda: abi.fp8_grouped_gemm_blockscaled(E, offs, Mrows, N, K, a, sa, w, sw,
+                                                          abi.MOE_EPI_BF16 | mode, out)
+        nbytes = E * N * K + Mrows * K + Mrows * (2 * N if args.case == "gemm2" else N // 2)
+        flops = 2 * Mrows * N * K
     elif args.case == "router":
         T, E2 = shape.T, shape.E
         x = synth.activations(T, H, 1, device=dev)
@@ -411,7 +426,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", default=None, help="time one kernel alone: gemm1 | gemm2 | router")
+    ap.add_argument("--case", default=None,
+                    help="time one kernel alone: gemm1 | gemm1_x256 | gemm1_skew | gemm2 | router")
+    ap.add_argument("--gemm-mode", default="auto", choices=["auto", "single", "pair"])
     args = ap.parse_args()
     if args.case:
         run_case(args)

@@ -71,7 +71,13 @@ enum moe_flag {
 enum moe_epilogue {
     MOE_EPI_BF16 = 0,          /* C bf16 [M, N]                                      */
     MOE_EPI_F32 = 1,           /* C fp32 [M, N]                                      */
-    MOE_EPI_SWIGLU_REQUANT = 2 /* N = 2I: C e4m3 [M, I] codes, sC fp32 [M, I/128]      */
+    MOE_EPI_SWIGLU_REQUANT = 2, /* N = 2I: C e4m3 [M, I] codes, sC fp32 [M, I/128]     */
+    /* OR-ed into `epilogue`: the tile mode.  Default (neither bit) and
+     * MOE_GEMM_SINGLE_CTA: one-SM tiles of 128 rows.  MOE_GEMM_PAIR_CTA: tiles
+     * of 256 rows on a cluster of two SMs (tcgen05 cta_group::2), each SM
+     * staging half of the weight tile.  Same results either way. */
+    MOE_GEMM_SINGLE_CTA = 0x100,
+    MOE_GEMM_PAIR_CTA = 0x200
 };
 
 /* Human-readable name of a moe_status value.  Static string, never NULL. */
@@ -159,8 +165,8 @@ int moe_permute(const moe_dims *dims, const int32_t *topk_idx, const uint8_t *xq
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture on the device.
- *   - Problems whose counts exceed the scratch (ceil(T/128) * E * 4 bytes >
- *     1 MiB, e.g. T > 131072 at E = 256) return MOE_ERR_TOO_LARGE.
+ *   - Problems whose counts exceed the scratch (ceil(T/32) * E * 4 bytes >
+ *     1 MiB, e.g. T > 32768 at E = 256) return MOE_ERR_TOO_LARGE.
  *   - All calls share the one array and it keeps the last call's contents;
  *     each call writes every count it reads before reading it, so nothing
  *     needs clearing.  Calls whose work overlaps on the GPU (different

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TOO_LARGE = range(6)
 MOE_FLAG_NONFINITE, MOE_FLAG_BAD_INDEX, MOE_FLAG_TIMEOUT, MOE_FLAG_BAD_OFFSETS = 1, 2, 4, 8
 MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_REQUANT = 0, 1, 2
+MOE_GEMM_SINGLE_CTA, MOE_GEMM_PAIR_CTA = 0x100, 0x200
 
 
 class MoEError(RuntimeError):

@@ -12,19 +12,32 @@
 // and add it to fp32 registers.  Two TMEM buffers (2 x 256 columns) let the
 // tensor core run block kb+1 while the epilogue promotes block kb.
 //
-// CTA organisation (persistent: one CTA per SM, 384 threads):
-//   warp 0        TMA producer: A tile 128x128 B + B tile 256x128 B per stage
-//   warp 1        TMEM allocator and MMA issuer (one elected lane)
+// Two variants share the code (template parameter PAIR):
+//   single  one CTA per SM, tile 128 rows x 256 columns; each stage holds the A
+//           tile (128 x 128 B) and the whole B tile (256 x 128 B).
+//   pair    clusters of two CTAs on two SMs share one tcgen05.mma.cta_group::2
+//           of M = 256: each CTA stages its own 128 rows of A and HALF of the
+//           B tile (128 of 256 rows), the leader CTA issues the MMA, and each
+//           CTA's TMEM receives its own 128 rows x 256 columns.  A weight tile is
+//           therefore streamed once for 256 rows, and each SM moves 32 KB per K
+//           block instead of 48 KB.  Transaction bytes of both CTAs' TMA loads and
+//           both CTAs' TMEM releases land on the leader's barriers; the leader's
+//           commits arrive on both CTAs' barriers.
+//
+// CTA organisation (persistent, 384 threads):
+//   warp 0        TMA producer
+//   warp 1        TMEM allocator and MMA issuer (one elected lane; the leader CTA
+//                 only in the pair variant)
 //   warps 2-3     idle (complete warpgroup 0 for setmaxnreg)
 //   warps 4-11    epilogue: warp w reads TMEM lanes 32*(w%4).., the two
 //                 warpgroups split the 256 accumulator columns
-// Tiles: 128 rows x 256 columns; the tile list (group-major, then N tile, then M
-// tile so that consecutive CTAs share a weight tile through L2) is derived on the
-// device from group_offsets, so no host synchronisation is needed.
+// The tile list (group-major, then N tile, then M tile so that CTAs working at
+// the same time share weight tiles through L2) is derived on the device from
+// group_offsets, so no host synchronisation is needed.
 //
-// No cluster launch and no multicast: every CTA loads its own tiles.  Every wait
-// is bounded (2 s); on expiry the CTA raises MOE_FLAG_TIMEOUT, drains its own
-// outstanding TMA loads and MMAs, frees its TMEM and returns.
+// No TMA multicast: every CTA loads its own tiles.  Every wait is bounded (2 s);
+// on expiry the CTA raises MOE_FLAG_TIMEOUT, drains its own outstanding TMA loads
+// and MMAs, frees its TMEM and returns.
 #include "tc_util.cuh"
 
 namespace moe {
@@ -32,32 +45,31 @@ namespace gg {
 
 using namespace moe::tc;
 
-constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;          // bytes == e4m3 elements == one 128B swizzle row
-constexpr int STAGES = 4;
-constexpr uint32_t A_BYTES = BM * BK;
+constexpr uint32_t A_BYTES = 128 * BK;
 constexpr uint32_t B_HALF = 128 * BK;
-constexpr uint32_t B_BYTES = BN * BK;
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 384;
 constexpr int EPI_THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAX_G = 4096;
 constexpr int LAUNCH_REGS = 168;   // 384 threads x 168 = 128 x 40 + 256 x 232
 
-// shared memory map (offsets from a 1024-aligned base)
-constexpr uint32_t OFF_STAGES = 0;
-constexpr uint32_t OFF_BARS = STAGES * STAGE_BYTES;                // 196608
-constexpr uint32_t OFF_MISC = OFF_BARS + 128;                      // tmem holder, abort, n_tiles, bad
-constexpr uint32_t OFF_RED = OFF_MISC + 32;                        // [2 parity][2 half][128] fp32
-constexpr uint32_t OFF_MSTART = OFF_RED + 2 * 2 * 128 * 4;         // int32 [MAX_G + 1]
-constexpr uint32_t SMEM_USED = OFF_MSTART + (MAX_G + 1) * 4;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;                  // + alignment slack
-
-// instruction descriptor: D fp32, A/B e4m3, K-major both, N = 256, M = 128
-constexpr uint32_t IDESC = (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
-                           (static_cast<uint32_t>(BM >> 4) << 24);
+template <bool PAIR>
+struct Cfg {
+    static constexpr int TM = PAIR ? 256 : 128;                     // rows per tile (whole pair)
+    static constexpr int STAGES = PAIR ? 6 : 4;
+    static constexpr uint32_t STAGE_BYTES = PAIR ? A_BYTES + B_HALF : A_BYTES + 2 * B_HALF;
+    static constexpr uint32_t OFF_BARS = STAGES * STAGE_BYTES;       // 196608 either way
+    static constexpr uint32_t OFF_MISC = OFF_BARS + 256;             // tmem holder, abort, bad
+    static constexpr uint32_t OFF_RED = OFF_MISC + 32;               // [2 parity][2 half][128] fp32
+    static constexpr uint32_t OFF_MSTART = OFF_RED + 2 * 2 * 128 * 4;  // int32 [MAX_G + 1]
+    static constexpr uint32_t SMEM_BYTES = OFF_MSTART + (MAX_G + 1) * 4 + 1024;
+    // instruction descriptor: D fp32, A/B e4m3, K-major both, N = 256, M = 128 or 256
+    static constexpr uint32_t IDESC = (1u << 4) | (static_cast<uint32_t>(BN >> 3) << 17) |
+                                      (static_cast<uint32_t>(TM >> 4) << 24);
+    static constexpr uint32_t TEMPTY_COUNT = PAIR ? 2 * EPI_THREADS : EPI_THREADS;
+};
 
 struct Tile {
     int g, m0, m_end, nt;
@@ -65,7 +77,7 @@ struct Tile {
 
 // Tile t -> (group, first row, group end, N tile).  Group g owns the tiles
 // [NT*mstart[g], NT*mstart[g+1]), ordered N-tile-major, M tile innermost.
-__device__ __forceinline__ Tile decode_tile(int t, const int32_t *mstart, int G, int NT,
+__device__ __forceinline__ Tile decode_tile(int t, const int32_t *mstart, int G, int NT, int TM,
                                             const int32_t *__restrict__ offs) {
     int lo = 0, hi = G;
     while (hi - lo > 1) {
@@ -78,16 +90,21 @@ __device__ __forceinline__ Tile decode_tile(int t, const int32_t *mstart, int G,
     r.g = lo;
     r.nt = local / mcount;
     const int mt = local % mcount;
-    r.m0 = __ldg(offs + lo) + mt * BM;
+    r.m0 = __ldg(offs + lo) + mt * TM;
     r.m_end = __ldg(offs + lo + 1);
     return r;
 }
 
+template <bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const int32_t *__restrict__ offs, int G, int64_t m_cap, int N, int K,
                     const float *__restrict__ sA, const float *__restrict__ sB, int epi,
                     void *__restrict__ C, float *__restrict__ sC, int32_t *status) {
+    using Cf = Cfg<PAIR>;
+    constexpr int STAGES = Cf::STAGES;
+    constexpr uint32_t STAGE_BYTES = Cf::STAGE_BYTES;
+    constexpr int TM = Cf::TM;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
     const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
@@ -95,7 +112,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const uint32_t sbase = raw_addr + pad;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t bar0 = sbase + OFF_BARS;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;   // 0 = leader of the pair
+    const bool leader = rank == 0;
+    const int unit = PAIR ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+    const int n_units = PAIR ? static_cast<int>(n_clusters_x()) : static_cast<int>(gridDim.x);
+
+    const uint32_t bar0 = sbase + Cf::OFF_BARS;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
     auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
@@ -103,11 +125,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
     auto xchg_bar = [&](int p) { return bar0 + 8u * (2 * STAGES + 5 + p); };
 
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
-    int *bad_flag = reinterpret_cast<int *>(smem + OFF_MISC + 8);
-    float *red = reinterpret_cast<float *>(smem + OFF_RED);
-    int32_t *mstart = reinterpret_cast<int32_t *>(smem + OFF_MSTART);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + Cf::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cf::OFF_MISC + 4);
+    int *bad_flag = reinterpret_cast<int *>(smem + Cf::OFF_MISC + 8);
+    float *red = reinterpret_cast<float *>(smem + Cf::OFF_RED);
+    int32_t *mstart = reinterpret_cast<int32_t *>(smem + Cf::OFF_MSTART);
 
     const bool swiglu = epi == MOE_EPI_SWIGLU_REQUANT;
     const int I = N / 2;
@@ -121,7 +143,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     for (int g = threadIdx.x; g < G; g += THREADS) {
         const int a = __ldg(offs + g), b = __ldg(offs + g + 1);
         if (b < a || a < 0 || static_cast<int64_t>(b) > m_cap) *bad_flag = 1;
-        mstart[g + 1] = b > a ? (b - a + BM - 1) / BM : 0;
+        mstart[g + 1] = b > a ? (b - a + TM - 1) / TM : 0;
     }
     __syncthreads();
     if (warp == 0) {
@@ -140,7 +162,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         if (lane == 0) mstart[0] = 0;
     } else if (warp == 2 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
-        for (int b = 0; b < 2; ++b) { mbar_init(tfull_bar(b), 1); mbar_init(tempty_bar(b), EPI_THREADS); }
+        for (int b = 0; b < 2; ++b) { mbar_init(tfull_bar(b), 1); mbar_init(tempty_bar(b), Cf::TEMPTY_COUNT); }
         mbar_init(drain_bar, 1);
         for (int p = 0; p < 2; ++p) mbar_init(xchg_bar(p), EPI_THREADS);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -150,18 +172,29 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
     if (warp == 1) {
         __syncwarp();
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         sbase + OFF_MISC),
-                     "r"(TMEM_COLS)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        if constexpr (PAIR) {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             sbase + Cf::OFF_MISC),
+                         "r"(TMEM_COLS)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             sbase + Cf::OFF_MISC),
+                         "r"(TMEM_COLS)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync();   // the peer's barriers and TMEM exist before any cross-CTA use
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
     const int num_tiles = *bad_flag ? 0 : NT * mstart[G];
     if (blockIdx.x == 0 && threadIdx.x == 0 && *bad_flag) set_flag(status, MOE_FLAG_BAD_OFFSETS);
+    // the leader's barriers as seen from this CTA (its own in the single variant)
+    const uint32_t lead_bar0 = PAIR ? mapa_shared(bar0, 0) : bar0;
 
     __syncwarp();
     if (warp < 4) {
@@ -174,52 +207,73 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             uint32_t phase = 0;
             int issued = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
-                const Tile tl = decode_tile(t, mstart, G, NT, offs);
-                const int r0 = swiglu ? 128 * tl.nt : BN * tl.nt;
-                const int r1 = swiglu ? I + 128 * tl.nt : BN * tl.nt + 128;
+            for (int t = unit; ok && t < num_tiles; t += n_units) {
+                const Tile tl = decode_tile(t, mstart, G, NT, TM, offs);
+                const int r0 = swiglu ? 128 * tl.nt : BN * tl.nt;            // B rows of columns 0..127
+                const int r1 = swiglu ? I + 128 * tl.nt : BN * tl.nt + 128;  // B rows of columns 128..255
+                const int arow = tl.m0 + 128 * static_cast<int>(rank);
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, status)) { ok = false; break; }
-                    const uint32_t sa = sbase + OFF_STAGES + stage * STAGE_BYTES;
-                    mbar_expect_tx(full_bar(stage), STAGE_BYTES);
-                    tma_load_2d(sa, &tmA, kb * BK, tl.m0, full_bar(stage));
-                    tma_load_3d(sa + A_BYTES, &tmB, kb * BK, r0, tl.g, full_bar(stage));
-                    tma_load_3d(sa + A_BYTES + B_HALF, &tmB, kb * BK, r1, tl.g, full_bar(stage));
+                    const uint32_t sa = sbase + stage * STAGE_BYTES;
+                    if constexpr (PAIR) {
+                        const uint32_t fb = lead_bar0 + 8u * stage;
+                        if (leader) mbar_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+                        tma_load_2d_pair(sa, &tmA, kb * BK, arow, fb);
+                        tma_load_3d_pair(sa + A_BYTES, &tmB, kb * BK, leader ? r0 : r1, tl.g, fb);
+                    } else {
+                        mbar_expect_tx(full_bar(stage), STAGE_BYTES);
+                        tma_load_2d(sa, &tmA, kb * BK, arow, full_bar(stage));
+                        tma_load_3d(sa + A_BYTES, &tmB, kb * BK, r0, tl.g, full_bar(stage));
+                        tma_load_3d(sa + A_BYTES + B_HALF, &tmB, kb * BK, r1, tl.g, full_bar(stage));
+                    }
                     ++issued;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
-            // no TMA write may land after this CTA exits: wait for the last loads
-            const int tail = issued < STAGES ? issued : STAGES;
-            for (int i = 0; i < tail; ++i) {
-                if (stage == 0) { stage = STAGES - 1; phase ^= 1u; } else { --stage; }
-                mbar_wait(full_bar(stage), phase, abort_flag, status, true);
+            // no TMA write may land after the CTAs exit: wait for the last loads
+            // (in a pair the leader's full barriers count both CTAs' bytes)
+            if (leader) {
+                const int tail = issued < STAGES ? issued : STAGES;
+                for (int i = 0; i < tail; ++i) {
+                    if (stage == 0) { stage = STAGES - 1; phase ^= 1u; } else { --stage; }
+                    mbar_wait(full_bar(stage), phase, abort_flag, status, true);
+                }
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && leader) {
             int stage = 0;
             uint32_t phase = 0, kc = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+            for (int t = unit; ok && t < num_tiles; t += n_units) {
                 for (int kb = 0; kb < KB; ++kb, ++kc) {
                     const uint32_t buf = kc & 1u, use = kc >> 1;
                     if (!mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
                     if (!mbar_wait(full_bar(stage), phase, abort_flag, status)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t sa = sbase + OFF_STAGES + stage * STAGE_BYTES;
+                    const uint32_t sa = sbase + stage * STAGE_BYTES;
                     const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sa + A_BYTES);
                     const uint32_t d = tmem_base + buf * 256u;
+                    if constexpr (PAIR) {
 #pragma unroll
-                    for (int k = 0; k < BK / 32; ++k) mma_f8(d, ad + 2u * k, bd + 2u * k, IDESC, k > 0 ? 1u : 0u);
-                    mma_commit(empty_bar(stage));
-                    mma_commit(tfull_bar(buf));
+                        for (int k = 0; k < BK / 32; ++k)
+                            mma_f8_pair(d, ad + 2u * k, bd + 2u * k, Cf::IDESC, k > 0 ? 1u : 0u);
+                        mma_commit_pair(empty_bar(stage), 0x3);
+                        mma_commit_pair(tfull_bar(buf), 0x3);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < BK / 32; ++k)
+                            mma_f8(d, ad + 2u * k, bd + 2u * k, Cf::IDESC, k > 0 ? 1u : 0u);
+                        mma_commit(empty_bar(stage));
+                        mma_commit(tfull_bar(buf));
+                    }
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
-            // every MMA of this CTA has completed before TMEM is released
-            mma_commit(drain_bar);
+            // every MMA of this CTA (pair) has completed before TMEM is released
+            if constexpr (PAIR) mma_commit_pair(drain_bar, 0x1);
+            else mma_commit(drain_bar);
             mbar_wait(drain_bar, 0, abort_flag, status, true);
         }
     }
@@ -233,12 +287,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         uint32_t kc = 0, xphase0 = 0, xphase1 = 0;
         int iter = 0;
         bool ok = true;
-        for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x, ++iter) {
-            const Tile tl = decode_tile(t, mstart, G, NT, offs);
-            const int64_t grow = static_cast<int64_t>(tl.m0) + row;
+        for (int t = unit; ok && t < num_tiles; t += n_units, ++iter) {
+            const Tile tl = decode_tile(t, mstart, G, NT, TM, offs);
+            const int64_t grow = static_cast<int64_t>(tl.m0) + 128 * static_cast<int>(rank) + row;
             const bool row_ok = grow < m_cap;
             const float *sa_row = sA + (row_ok ? grow : 0) * KB;
-            // per-chunk TMEM column and scale row of B
+            // scale rows of B for the two column halves of this thread
             int nb0, nb1;
             bool nb1_ok = true;
             if (swiglu) { nb0 = tl.nt; nb1 = I / 128 + tl.nt; }
@@ -264,11 +318,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     uint32_t r[32];
                     tmem_ld32(lane_base + buf * 256u + col, r);
                     const float sc = (swiglu && c >= 2) ? s1 : s0;
+                    const float2 sc2 = make_float2(sc, sc);
+                    // packed dual fp32 FMA: the same round-to-nearest FMA per element, half the issues
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) acc[32 * c + j] = fmaf(sc, __uint_as_float(r[j]), acc[32 * c + j]);
+                    for (int j = 0; j < 32; j += 2) {
+                        const float2 a2 = __ffma2_rn(sc2, make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
+                                                     make_float2(acc[32 * c + j], acc[32 * c + j + 1]));
+                        acc[32 * c + j] = a2.x;
+                        acc[32 * c + j + 1] = a2.y;
+                    }
                 }
                 tc_fence_before();
-                mbar_arrive(tempty_bar(buf));
+                if constexpr (PAIR) mbar_arrive_cluster(lead_bar0 + 8u * (2 * STAGES + 2 + buf));
+                else mbar_arrive(tempty_bar(buf));
             }
             if (!ok) break;
             const bool store_row = grow < tl.m_end;
@@ -344,29 +406,61 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
     tc_fence_before();
     __syncthreads();
+    // the leader's MMAs into the peer's TMEM, the peer's TMA bytes and TMEM
+    // releases on the leader's barriers: all done before either CTA frees or exits
+    if constexpr (PAIR) cluster_sync();
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
-                     : "memory");
+        if constexpr (PAIR)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                         : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                         : "memory");
     }
 }
 
-
+template <bool PAIR>
 static int prepare_kernel() {
     static int state = 0;   // 0 unknown, 1 ready, 2 unsupported
     if (state == 0) {
         cudaFuncAttributes attr;
-        if (cudaFuncGetAttributes(&attr, grouped_gemm_kernel) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaFuncGetAttributes(&attr, grouped_gemm_kernel<PAIR>) != cudaSuccess) return MOE_ERR_CUDA;
         // setmaxnreg moves registers inside the launch's allotment: the split
         // 128 x 40 + 256 x 232 must equal 384 x (registers at launch)
         if (attr.numRegs != LAUNCH_REGS) { state = 2; return MOE_ERR_UNSUPPORTED; }
-        if (cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(SMEM_BYTES)) != cudaSuccess)
+        if (cudaFuncSetAttribute(grouped_gemm_kernel<PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(Cfg<PAIR>::SMEM_BYTES)) != cudaSuccess)
             return MOE_ERR_CUDA;
         state = 1;
     }
     return state == 1 ? MOE_OK : MOE_ERR_UNSUPPORTED;
+}
+
+// Co-resident CTA pairs for one wave of the persistent pair kernel.
+static int pair_clusters(cudaStream_t st) {
+    static int cached = 0;
+    if (cached == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(num_sms() / 2 * 2), 1, 1);
+        cfg.blockDim = dim3(THREADS, 1, 1);
+        cfg.dynamicSmemBytes = Cfg<true>::SMEM_BYTES;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<true>, &cfg) == cudaSuccess && n > 0)
+            cached = n;
+        else
+            cached = num_sms() / 2;
+    }
+    return cached;
 }
 
 }  // namespace gg
@@ -379,6 +473,10 @@ MOE_API int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets
                                          const uint8_t *B, const float *sB, int32_t epilogue, void *C,
                                          float *sC, int32_t *status, void *stream) {
     using namespace moe::gg;
+    // tile mode: one-SM tiles unless CTA pairs are asked for (measured on B200:
+    // pairs are no faster at the shapes of this layer)
+    const bool single = (epilogue & MOE_GEMM_PAIR_CTA) == 0 || (epilogue & MOE_GEMM_SINGLE_CTA) != 0;
+    epilogue &= ~(MOE_GEMM_SINGLE_CTA | MOE_GEMM_PAIR_CTA);
     if (G < 0 || m_capacity < 0 || N < 0 || K < 0) return MOE_ERR_INVALID_ARG;
     if (N % 128 != 0 || K % 128 != 0) return MOE_ERR_INVALID_ARG;
     if (epilogue != MOE_EPI_BF16 && epilogue != MOE_EPI_F32 && epilogue != MOE_EPI_SWIGLU_REQUANT)
@@ -391,7 +489,7 @@ MOE_API int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets
     if (!aligned16(A) || !aligned16(B) || !aligned16(C) || (reinterpret_cast<uintptr_t>(sA) & 3) ||
         (reinterpret_cast<uintptr_t>(sB) & 3) || (sC && (reinterpret_cast<uintptr_t>(sC) & 3)))
         return MOE_ERR_INVALID_ARG;
-    int rc = prepare_kernel();
+    int rc = single ? prepare_kernel<false>() : prepare_kernel<true>();
     if (rc != MOE_OK) return rc;
     auto enc = encode_fn();
     if (!enc) return MOE_ERR_CUDA;
@@ -417,9 +515,27 @@ MOE_API int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return MOE_ERR_CUDA;
     }
-    const int grid = num_sms();
-    grouped_gemm_kernel<<<grid, THREADS, SMEM_BYTES, as_stream(stream)>>>(
-        tmA, tmB, group_offsets, G, m_capacity, static_cast<int>(N), static_cast<int>(K), sA, sB, epilogue, C,
-        sC, status);
+    cudaStream_t st = as_stream(stream);
+    const int n = static_cast<int>(N), k = static_cast<int>(K);
+    if (single) {
+        grouped_gemm_kernel<false><<<num_sms(), THREADS, Cfg<false>::SMEM_BYTES, st>>>(
+            tmA, tmB, group_offsets, G, m_capacity, n, k, sA, sB, epilogue, C, sC, status);
+        return launch_status();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pair_clusters(st)), 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = Cfg<true>::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<true>, tmA, tmB, group_offsets, G, m_capacity, n, k, sA, sB,
+                           static_cast<int>(epilogue), C, sC, status) != cudaSuccess)
+        return MOE_ERR_CUDA;
     return launch_status();
 }

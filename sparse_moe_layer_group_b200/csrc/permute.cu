@@ -18,7 +18,7 @@
 
 namespace moe {
 
-constexpr int PERM_CHUNK = 128;
+constexpr int PERM_CHUNK = 32;
 constexpr int PERM_MAX_E = 1024;
 
 __global__ void perm_count_kernel(const int32_t *__restrict__ idx, int32_t *__restrict__ counts, int T,
@@ -177,7 +177,7 @@ MOE_API int moe_permute(const moe_dims *d, const int32_t *topk_idx, const uint8_
 
 namespace moe {
 
-constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(1) << 20;   // 1 MiB: counts[n_chunks][E] int32
+constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(1) << 20;   // 1 MiB: counts[ceil(T/32)][E] int32
 constexpr int NOALLOC_MAX_DEVICES = 64;
 
 static __device__ __align__(256) int32_t g_perm_noalloc_scratch[NOALLOC_SCRATCH_BYTES / sizeof(int32_t)];

@@ -12,23 +12,24 @@
 
 namespace moe {
 
-// 16 lanes own one 1x128 tile: lane l holds columns 8l .. 8l+7.
-__global__ void __launch_bounds__(256) quant_1x128_kernel(const uint4 *__restrict__ x,
-                                                          uint2 *__restrict__ q,
-                                                          float *__restrict__ scales,
-                                                          int64_t n_tiles, int32_t *status) {
-    const int lane16 = threadIdx.x & 15;
-    const int64_t half_id = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
-    const int64_t n_halves = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 4;
-    // every 16-lane half runs the same trip count so the shuffles stay converged
-    const int64_t trips = (n_tiles + n_halves - 1) / n_halves;
-    for (int64_t it = 0; it < trips; ++it) {
-        const int64_t tile = half_id + it * n_halves;
-        const bool live = tile < n_tiles;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (live) v = __ldg(x + tile * 16 + lane16);
-        float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                      bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+// 16 lanes own one 1x128 tile: lane l holds columns 8l .. 8l+7.  Each trip
+// handles Q tiles per half-warp with all Q loads issued first, so several
+// 16-byte loads per thread are in flight.
+template <int Q>
+__device__ __forceinline__ void quant_tiles(const uint4 *__restrict__ x, uint2 *__restrict__ q,
+                                            float *__restrict__ scales, int64_t first, int64_t stride,
+                                            int64_t n_tiles, int lane16, int32_t *status) {
+    uint4 v[Q];
+#pragma unroll
+    for (int u = 0; u < Q; ++u) {
+        const int64_t tile = first + u * stride;
+        v[u] = tile < n_tiles ? __ldg(x + tile * 16 + lane16) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < Q; ++u) {
+        const int64_t tile = first + u * stride;
+        const float f[8] = {bf16_lo(v[u].x), bf16_hi(v[u].x), bf16_lo(v[u].y), bf16_hi(v[u].y),
+                            bf16_lo(v[u].z), bf16_hi(v[u].z), bf16_lo(v[u].w), bf16_hi(v[u].w)};
         float amax = 0.0f;
         bool fin = true;
 #pragma unroll
@@ -39,20 +40,36 @@ __global__ void __launch_bounds__(256) quant_1x128_kernel(const uint4 *__restric
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
             fin_i &= __shfl_xor_sync(0xffffffffu, fin_i, o);
         }
-        if (!live) continue;
+        if (tile >= n_tiles) continue;
         const bool finite = fin_i != 0;
-        const float s = tile_scale(amax, finite);
+        const float sc = tile_scale(amax, finite);
         uint32_t lo = 0, hi = 0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) lo |= static_cast<uint32_t>(quant_code(f[i], s, finite)) << (8 * i);
+        for (int i = 0; i < 4; ++i) lo |= static_cast<uint32_t>(quant_code(f[i], sc, finite)) << (8 * i);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) hi |= static_cast<uint32_t>(quant_code(f[4 + i], s, finite)) << (8 * i);
+        for (int i = 0; i < 4; ++i) hi |= static_cast<uint32_t>(quant_code(f[4 + i], sc, finite)) << (8 * i);
         q[tile * 16 + lane16] = make_uint2(lo, hi);
         if (lane16 == 0) {
-            scales[tile] = s;
+            scales[tile] = sc;
             if (!finite) set_flag(status, MOE_FLAG_NONFINITE);
         }
     }
+}
+
+constexpr int QUANT_Q = 4;
+
+__global__ void __launch_bounds__(256) quant_1x128_kernel(const uint4 *__restrict__ x,
+                                                          uint2 *__restrict__ q,
+                                                          float *__restrict__ scales,
+                                                          int64_t n_tiles, int32_t *status) {
+    const int lane16 = threadIdx.x & 15;
+    const int64_t half_id = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
+    const int64_t n_halves = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 4;
+    // every 16-lane half runs the same trip count so the shuffles stay converged
+    const int64_t per_trip = n_halves * QUANT_Q;
+    const int64_t trips = (n_tiles + per_trip - 1) / per_trip;
+    for (int64_t it = 0; it < trips; ++it)
+        quant_tiles<QUANT_Q>(x, q, scales, half_id + it * per_trip, n_halves, n_tiles, lane16, status);
 }
 
 // One CTA per 128x128 block: 256 threads, each row of the block is 16 lanes x 16 B.
@@ -164,8 +181,8 @@ MOE_API int fp8_quant_1x128(const void *x, int64_t rows, int64_t cols, uint8_t *
     if (!x || !q || !scales || !aligned16(x) || !aligned16(q) || !aligned16(scales))
         return MOE_ERR_INVALID_ARG;
     const int64_t n_tiles = rows * (cols / 128);
-    const int64_t halves_per_block = 256 / 16;
-    int64_t blocks = (n_tiles + halves_per_block - 1) / halves_per_block;
+    const int64_t tiles_per_block = 256 / 16 * QUANT_Q;
+    int64_t blocks = (n_tiles + tiles_per_block - 1) / tiles_per_block;
     const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
     if (blocks > cap) blocks = cap;
     quant_1x128_kernel<<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(

@@ -151,8 +151,10 @@ class MoELayer:
                         self.out_f32 if out_f32 else None, stream)
         return self.out
 
-    def bias_update(self, gamma: float, stream=None):
-        abi.moe_bias_update(self.E, self.T, self.K, gamma, self.load, self.e_bias, stream)
+    def bias_update(self, gamma: float, stream=None, bias: Optional[torch.Tensor] = None):
+        """b += gamma * sign(T*K/E - load) from this step's expert loads, into
+        the routing bias (default) or into `bias` (keeps the routing fixed)."""
+        abi.moe_bias_update(self.E, self.T, self.K, gamma, self.load, self.e_bias if bias is None else bias, stream)
 
     # ---- algorithmic work of one forward (for throughput and roofline figures)
     def flops(self) -> dict:

@@ -46,12 +46,17 @@ GEMM_CASES = [  # sizes, N, K
     ([5] * 40, 256, 384),                       # many small groups
     (list(range(0, 300, 7)), 768, 512),         # 43 groups, > 148 tiles: persistent loop
     ([128, 128, 256], 256, 128),                # exact tiles, single K block
+    ([600, 0, 255, 256, 1], 512, 384),          # several 256-row pair tiles, ragged
 ]
+
+
+TILE_MODES = {"pair": 0x200, "single": 0x100}   # CTA-pair tiles or one-SM tiles
 
 
 @pytest.mark.parametrize("sizes,N,K", GEMM_CASES)
 @pytest.mark.parametrize("epi", ["f32", "bf16"])
-def test_grouped_gemm(lib, sizes, N, K, epi):
+@pytest.mark.parametrize("mode", list(TILE_MODES))
+def test_grouped_gemm(lib, sizes, N, K, epi, mode):
     a, b, aq, sa, bq, sb, offs, M = _operands(sizes, N, K, seed=len(sizes) * 7 + N + K, m_extra=3)
     qa, qsa, qb, qsb = _gpu_operands(lib, a, b)
     ref = oracle.grouped_gemm_blockscaled(offs, aq, sa, bq, sb)
@@ -59,8 +64,9 @@ def test_grouped_gemm(lib, sizes, N, K, epi):
     sentinel = 7.0
     C = torch.full((M, N), sentinel, dtype=dt, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    e = (lib.MOE_EPI_F32 if epi == "f32" else lib.MOE_EPI_BF16) | TILE_MODES[mode]
     lib.fp8_grouped_gemm_blockscaled(len(sizes), cuda(torch.from_numpy(offs)), M, N, K, qa, qsa, qb, qsb,
-                                     lib.MOE_EPI_F32 if epi == "f32" else lib.MOE_EPI_BF16, C, None, st)
+                                     e, C, None, st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     got = np_(C)
@@ -75,7 +81,8 @@ def test_grouped_gemm(lib, sizes, N, K, epi):
     assert np.all(np.abs(g - r) <= tol)
 
 
-def test_integer_exact_gemm(lib):
+@pytest.mark.parametrize("mode", list(TILE_MODES))
+def test_integer_exact_gemm(lib, mode):
     """Integer-valued codes with unit-friendly scales: the result is an exact
     integer matrix on both sides (fp32 sums of integers below 2^24)."""
     rng = np.random.default_rng(0)
@@ -91,14 +98,16 @@ def test_integer_exact_gemm(lib):
     assert torch.all(qsa == 1.0) and torch.all(qsb == 1.0)
     C = torch.empty(M, N, dtype=torch.float32, device="cuda")
     offs = torch.tensor([0, M], dtype=torch.int32, device="cuda")
-    lib.fp8_grouped_gemm_blockscaled(1, offs, M, N, K, qa, qsa, qb, qsb, lib.MOE_EPI_F32, C)
+    lib.fp8_grouped_gemm_blockscaled(1, offs, M, N, K, qa, qsa, qb, qsb, lib.MOE_EPI_F32 | TILE_MODES[mode], C)
     torch.cuda.synchronize()
     exact = ai.astype(np.int64) @ bi.astype(np.int64).T
     assert np.array_equal(np_(C).astype(np.int64), exact)
 
 
-@pytest.mark.parametrize("sizes,I,K", [([70, 0, 150], 256, 384), ([1], 128, 128), ([300] * 3, 512, 1024)])
-def test_grouped_gemm_swiglu_requant(lib, sizes, I, K):
+@pytest.mark.parametrize("sizes,I,K", [([70, 0, 150], 256, 384), ([1], 128, 128), ([300] * 3, 512, 1024),
+                                       ([257, 511, 3, 0, 129], 256, 256)])
+@pytest.mark.parametrize("mode", list(TILE_MODES))
+def test_grouped_gemm_swiglu_requant(lib, sizes, I, K, mode):
     N = 2 * I
     a, b, aq, sa, bq, sb, offs, M = _operands(sizes, N, K, seed=91 + I, heavy=False)
     qa, qsa, qb, qsb = _gpu_operands(lib, a, b)
@@ -106,7 +115,7 @@ def test_grouped_gemm_swiglu_requant(lib, sizes, I, K):
     s = torch.empty(M, I // 128, dtype=torch.float32, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     lib.fp8_grouped_gemm_blockscaled(len(sizes), cuda(torch.from_numpy(offs)), M, N, K, qa, qsa, qb, qsb,
-                                     lib.MOE_EPI_SWIGLU_REQUANT, q, s, st)
+                                     lib.MOE_EPI_SWIGLU_REQUANT | TILE_MODES[mode], q, s, st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     gu = oracle.grouped_gemm_blockscaled(offs, aq, sa, bq, sb)
@@ -124,7 +133,8 @@ def test_grouped_gemm_swiglu_requant(lib, sizes, I, K):
     assert normwise(deq_g, act) < 0.05
 
 
-def test_bad_offsets_flagged(lib):
+@pytest.mark.parametrize("mode", list(TILE_MODES))
+def test_bad_offsets_flagged(lib, mode):
     M, N, K = 64, 256, 128
     qa = torch.zeros(M, K, dtype=torch.uint8, device="cuda")
     qsa = torch.ones(M, 1, dtype=torch.float32, device="cuda")
@@ -133,7 +143,8 @@ def test_bad_offsets_flagged(lib):
     C = torch.full((M, N), 3.0, dtype=torch.float32, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     offs = torch.tensor([0, 40, 20], dtype=torch.int32, device="cuda")   # decreasing
-    lib.fp8_grouped_gemm_blockscaled(2, offs, M, N, K, qa, qsa, qb, qsb, lib.MOE_EPI_F32, C, None, st)
+    lib.fp8_grouped_gemm_blockscaled(2, offs, M, N, K, qa, qsa, qb, qsb, lib.MOE_EPI_F32 | TILE_MODES[mode], C,
+                                     None, st)
     torch.cuda.synchronize()
     assert int(st.item()) & lib.MOE_FLAG_BAD_OFFSETS
     assert torch.all(C == 3.0)

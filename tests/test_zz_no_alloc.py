@@ -53,7 +53,7 @@ def test_noalloc_rejects_problems_beyond_its_scratch(lib):
     cap = lib.abi.moe_permute_noalloc_max_scratch()
     assert cap == 1 << 20
     E = 256
-    T = (cap // (4 * E)) * 128 + 1           # one chunk too many
+    T = (cap // (4 * E)) * 32 + 1            # one 32-token chunk too many
     d = lib.dims(T, 128, E, 8, 1, 1, 128, 2.5)
     with pytest.raises(lib.MoEError) as ei:
         lib.abi.moe_permute_noalloc(d, None, None, None, None, None, None, None, None, None)
