@@ -36,7 +36,7 @@ function is "parity unpinned".
 from .fp8 import (E4M3_MAX, e4m3_encode, e4m3_decode, e4m3_encode_scalar, e4m3_decode_scalar,
                   round_bf16, quant_1x128, quant_128x128, dequant_1x128, dequant_128x128)
 from .routing import (router_scores, select_experts, select_experts_bruteforce,
-                      expert_load, bias_update)
+                      expert_load, bias_update, seq_balance_loss, load_entropy)
 from .dispatch import permute, unpermute_rows, combine
 from .expert import (gemm_blockscaled, grouped_gemm_blockscaled, silu, swiglu,
                      swiglu_requant, expert_ffn)
@@ -46,6 +46,7 @@ __all__ = [
     "E4M3_MAX", "e4m3_encode", "e4m3_decode", "e4m3_encode_scalar", "e4m3_decode_scalar",
     "round_bf16", "quant_1x128", "quant_128x128", "dequant_1x128", "dequant_128x128",
     "router_scores", "select_experts", "select_experts_bruteforce", "expert_load", "bias_update",
+    "seq_balance_loss", "load_entropy",
     "permute", "unpermute_rows", "combine",
     "gemm_blockscaled", "grouped_gemm_blockscaled", "silu", "swiglu", "swiglu_requant", "expert_ffn",
     "LayerWeights", "quantize_layer_weights", "moe_forward", "moe_forward_tokens",

@@ -136,3 +136,40 @@ def bias_update(bias32, load, T: int, K: int, gamma: float) -> np.ndarray:
         elif diff < 0:      # over-loaded: lower it
             b[e] = np.float32(b[e] - g32)
     return b
+
+
+def seq_balance_loss(s, idx, seq_len: int, alpha: float) -> np.ndarray:
+    """Sequence-wise balance loss, one value per sequence ([report-walkthrough]
+    section 3.3: per sequence, the sum over experts of each expert's share of the
+    sequence's assignments times its mean affinity over the sequence, times a
+    small coefficient alpha; aux_loss_alpha 0.001 in [repro-guide] section 3).
+
+    Reading (the pages give no normalisation): for a sequence of S tokens,
+        f_i = (#slots of the sequence routed to i) / (S * K)
+        P_i = (1 / S) * sum_t s[t, i]        (the sigmoid affinities)
+        L   = alpha * sum_i f_i * P_i
+    s [T, E] affinities, idx [T, K]; T must be a multiple of seq_len.
+    Returns float64 [T / seq_len]."""
+    s = np.asarray(s, dtype=np.float64)
+    idx = np.asarray(idx, dtype=np.int64)
+    T, E = s.shape
+    K = idx.shape[1]
+    assert T % seq_len == 0
+    out = np.zeros(T // seq_len)
+    for q in range(T // seq_len):
+        rows = slice(q * seq_len, (q + 1) * seq_len)
+        f = np.bincount(idx[rows].reshape(-1), minlength=E) / (seq_len * K)
+        P = s[rows].sum(axis=0) / seq_len
+        out[q] = alpha * float(np.sum(f * P))
+    return out
+
+
+def load_entropy(load) -> float:
+    """Entropy (natural log) of the expert-load distribution p_i = load_i / sum(load),
+    with 0 log 0 = 0: log(E) for perfectly even loads, 0 when one expert takes all."""
+    load = np.asarray(load, dtype=np.float64)
+    tot = load.sum()
+    if tot <= 0:
+        return 0.0
+    p = load[load > 0] / tot
+    return float(-np.sum(p * np.log(p)))

@@ -120,3 +120,39 @@ def test_load_and_bias_update_hand_computed():
     # the mean need not be an integer: T*K/E = 3/2 -> load 1 under, load 2 over
     nb3 = oracle.bias_update(np.zeros(2, np.float32), np.array([1, 2]), 3, 1, 0.5)
     assert list(nb3) == [0.5, -0.5]
+
+
+def test_seq_balance_loss_hand_computed():
+    # one sequence of 2 tokens, E = 2, K = 1: token 0 -> expert 0, token 1 -> expert 0
+    s = np.array([[0.8, 0.2], [0.6, 0.4]])
+    idx = np.array([[0], [0]])
+    # f = (1, 0), P = (0.7, 0.3): L = alpha * 0.7
+    assert np.allclose(oracle.seq_balance_loss(s, idx, 2, 0.001), [0.0007], rtol=1e-15)
+    # two sequences of one token each
+    got = oracle.seq_balance_loss(s, np.array([[0], [1]]), 1, 1.0)
+    assert np.allclose(got, [0.8, 0.4], rtol=1e-15)
+
+
+def test_seq_balance_loss_closed_forms():
+    # constant affinities c and any routing: sum_i f_i = 1, so L = alpha * c
+    T, E, K = 64, 16, 4
+    idx = synth.topk_indices(T, E, K, 3).numpy()
+    s = np.full((T, E), 0.25)
+    assert np.allclose(oracle.seq_balance_loss(s, idx, 16, 0.01), 0.0025, rtol=1e-14)
+    # against a brute-force triple loop
+    s = synth.scores(T, E, 9).numpy().astype(np.float64)
+    want = []
+    for q in range(4):
+        acc = 0.0
+        for i in range(E):
+            cnt = sum(1 for t in range(16 * q, 16 * q + 16) for k in range(K) if idx[t, k] == i)
+            mean = sum(s[t, i] for t in range(16 * q, 16 * q + 16)) / 16
+            acc += cnt / (16 * K) * mean
+        want.append(0.001 * acc)
+    assert np.allclose(oracle.seq_balance_loss(s, idx, 16, 0.001), want, rtol=1e-13)
+
+
+def test_load_entropy_closed_forms():
+    assert abs(oracle.load_entropy(np.full(256, 128)) - np.log(256)) < 1e-12
+    assert oracle.load_entropy(np.array([0, 0, 5, 0])) == 0.0
+    assert abs(oracle.load_entropy(np.array([1, 1, 2])) - (-(0.25 * np.log(0.25) * 2 + 0.5 * np.log(0.5)))) < 1e-15
