@@ -214,6 +214,10 @@ def run_gpu(args, rank, world, local):
     g1_ms = sum(a.elapsed_time(b) for a, b in g1_events) / len(g1_events)
     load = layer.load.cpu().numpy()
     touched = int((load > 0).sum())
+    seq_loss, entropy = layer.balance_stats(T, 0.001)     # one 4096-token sequence per step
+    balance = {"max_over_mean_load": round(float(load.max() / load.mean()), 3),
+               "load_entropy": round(float(entropy.item()), 5), "uniform_entropy": round(float(np.log(layer.E)), 5),
+               "seq_balance_loss": float(seq_loss[0].item())}
 
     # end to end through the public API: pinned host input, copy in, forward,
     # copy the output back, every step
@@ -277,6 +281,7 @@ def run_gpu(args, rank, world, local):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "device_status": status,
+        "balance": balance,
     }
     return rec
 

@@ -219,6 +219,22 @@ int swiglu_requant(const float *gu, int64_t M, int64_t I, uint8_t *q, float *s, 
 int moe_combine(const moe_dims *dims, const void *yperm, const int32_t *row_of,
                 const float *topk_w, const void *yshared, void *out, float *out_f32, void *stream);
 
+/* Sequence-wise balance loss and expert-load entropy ([report-walkthrough]
+ * section 3.3: a complementary per-sequence balance loss with a very small
+ * coefficient; aux_loss_alpha 0.001 in [repro-guide] section 3).  For each
+ * sequence q of seq_len tokens (T % seq_len == 0):
+ *   f_i = (#slots of the sequence routed to i) / (seq_len * K)
+ *   P_i = mean over the sequence's tokens of scores[t, i]
+ *   seq_loss[q] = alpha * sum_i f_i * P_i                    float64 [T/seq_len]
+ *   *entropy = -sum_i p_i ln p_i, p_i = expert_load[i] / sum(expert_load)
+ * Sums are float64 in a fixed order (deterministic).  seq_loss or entropy may
+ * be NULL to skip that output.
+ *   scores fp32 [T, E] (moe_route's affinities), topk_idx int32 [T, K],
+ *   expert_load int32 [E] (moe_permute's load).                                */
+int moe_balance_stats(const moe_dims *dims, const float *scores, const int32_t *topk_idx,
+                      const int32_t *expert_load, int32_t seq_len, double alpha, double *seq_loss,
+                      double *entropy, void *stream);
+
 /* Auxiliary-loss-free bias update ([report-walkthrough] section 3.2; rate
  * expert_bias_update_rate 0.001 in [repro-guide] section 3):
  *   e_bias[e] += gamma * sign(T*K/E - expert_load[e]),  sign(0) = 0,

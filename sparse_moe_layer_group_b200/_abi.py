@@ -62,6 +62,7 @@ _SIGS = {
     "swiglu_requant": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P]),
     "moe_combine": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P]),
     "moe_bias_update": (ctypes.c_int, [_I32, _I64, _I32, _F, _P, _P, _P]),
+    "moe_balance_stats": (ctypes.c_int, [_DIMS, _P, _P, _P, _I32, ctypes.c_double, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -178,3 +179,9 @@ def moe_combine(d, yperm, row_of, topk_w, yshared, out, out_f32=None, stream=Non
 def moe_bias_update(E, T, K, gamma, expert_load, e_bias, stream=None):
     _check("moe_bias_update", _lib.moe_bias_update(int(E), int(T), int(K), float(gamma), _ptr(expert_load),
                                                    _ptr(e_bias), _stream(stream)))
+
+
+def moe_balance_stats(d, scores, topk_idx, expert_load, seq_len, alpha, seq_loss, entropy, stream=None):
+    _check("moe_balance_stats", _lib.moe_balance_stats(ctypes.byref(d), _ptr(scores), _ptr(topk_idx),
+                                                       _ptr(expert_load), int(seq_len), float(alpha),
+                                                       _ptr(seq_loss), _ptr(entropy), _stream(stream)))

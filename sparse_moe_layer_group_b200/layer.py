@@ -156,6 +156,14 @@ class MoELayer:
         the routing bias (default) or into `bias` (keeps the routing fixed)."""
         abi.moe_bias_update(self.E, self.T, self.K, gamma, self.load, self.e_bias if bias is None else bias, stream)
 
+    def balance_stats(self, seq_len: int, alpha: float = 0.001, stream=None):
+        """(per-sequence balance loss float64 [T/seq_len], load entropy float64 [1])
+        of the last forward, computed on the device."""
+        loss = torch.empty(self.T // seq_len, dtype=torch.float64, device=self.out.device)
+        ent = torch.empty(1, dtype=torch.float64, device=self.out.device)
+        abi.moe_balance_stats(self.d, self.scores, self.topk_idx, self.load, seq_len, alpha, loss, ent, stream)
+        return loss, ent
+
     # ---- algorithmic work of one forward (for throughput and roofline figures)
     def flops(self) -> dict:
         T, H, K, I = self.T, self.H, self.K, self.I

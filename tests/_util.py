@@ -31,3 +31,33 @@ def bf16_ulp(v) -> np.ndarray:
 
 def cuda(t: torch.Tensor) -> torch.Tensor:
     return t.contiguous().cuda()
+
+
+def router_logit_tol(x, w_router, pieces: int = 3):
+    """Per-token bound on the router-logit error of an fp32 accumulation of the
+    H-term dot products (computed as `pieces` * H exact products): a random walk
+    of per-add roundings of at most half an fp32 ulp of the running magnitude,
+    taken at 8 standard deviations, with the running magnitude bounded by
+    sum_h |x_h w_eh| (the largest over experts).  Returns float64 [T]."""
+    x64 = np.abs(np.asarray(x, dtype=np.float64))
+    w64 = np.abs(np.asarray(w_router, dtype=np.float64))
+    mag = (x64 @ w64.T).max(axis=1)
+    n = pieces * x64.shape[1]
+    return 8.0 * np.sqrt(n) * 2.0 ** -24 * mag
+
+
+def same_expert_sets(idx_a, idx_b):
+    """Per token: the two routing tables select the same set of experts."""
+    a = np.sort(np.asarray(idx_a), axis=1)
+    b = np.sort(np.asarray(idx_b), axis=1)
+    return np.all(a == b, axis=1)
+
+
+def order_is_valid(idx, s32, b32):
+    """Per token: the table lists its experts by descending s + b (fp32), ties
+    to the lower index -- the order rule, checked on the given affinities."""
+    idx = np.asarray(idx, dtype=np.int64)
+    r = (np.asarray(s32, dtype=np.float32) + np.asarray(b32, dtype=np.float32)).astype(np.float32)
+    v = np.take_along_axis(r, idx, axis=1).astype(np.float64)
+    ok = (v[:, :-1] > v[:, 1:]) | ((v[:, :-1] == v[:, 1:]) & (idx[:, :-1] < idx[:, 1:]))
+    return np.all(ok, axis=1)
