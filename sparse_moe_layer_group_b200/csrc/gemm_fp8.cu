@@ -58,9 +58,9 @@ constexpr int LAUNCH_REGS = 168;   // 384 threads x 168 = 128 x 40 + 256 x 232
 template <bool PAIR>
 struct Cfg {
     static constexpr int TM = PAIR ? 256 : 128;                     // rows per tile (whole pair)
-    static constexpr int STAGES = PAIR ? 6 : 4;
+    static constexpr int STAGES = PAIR ? 6 : 3;     // 3 x 48 KB: a fourth stage measured no faster
     static constexpr uint32_t STAGE_BYTES = PAIR ? A_BYTES + B_HALF : A_BYTES + 2 * B_HALF;
-    static constexpr uint32_t OFF_BARS = STAGES * STAGE_BYTES;       // 196608 either way
+    static constexpr uint32_t OFF_BARS = STAGES * STAGE_BYTES;
     static constexpr uint32_t OFF_MISC = OFF_BARS + 256;             // tmem holder, abort, bad
     static constexpr uint32_t OFF_RED = OFF_MISC + 32;               // [2 parity][2 half][128] fp32
     static constexpr uint32_t OFF_MSTART = OFF_RED + 2 * 2 * 128 * 4;  // int32 [MAX_G + 1]

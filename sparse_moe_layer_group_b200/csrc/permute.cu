@@ -40,32 +40,72 @@ __global__ void perm_count_kernel(const int32_t *__restrict__ idx, int32_t *__re
     }
 }
 
-// One CTA of up to 1024 threads.
-__global__ void perm_scan_kernel(int32_t *__restrict__ counts, int n_chunks, int E,
-                                 int32_t *__restrict__ load, int32_t *__restrict__ offsets) {
+// One CTA of SCAN_THREADS threads.  Thread (p, e) owns expert e's chunks
+// [p*n/P, (p+1)*n/P): pass 1 sums them (loads batched), the P partial sums of
+// each expert are scanned in shared memory, pass 2 writes the exclusive
+// per-chunk prefixes.  Then the per-expert totals are scanned into offsets.
+constexpr int SCAN_THREADS = 1024;
+
+__global__ void __launch_bounds__(SCAN_THREADS) perm_scan_kernel(int32_t *__restrict__ counts, int n_chunks,
+                                                                 int E, int P, int32_t *__restrict__ load,
+                                                                 int32_t *__restrict__ offsets) {
+    __shared__ int32_t part[SCAN_THREADS];
     __shared__ int32_t sums[PERM_MAX_E];
-    const int e = threadIdx.x;
-    int run = 0;
+    const int tid = threadIdx.x;
+    const int Ep = blockDim.x / P;             // experts per pass (>= E)
+    const int e = tid % Ep, p = tid / Ep;
+    const int per = (n_chunks + P - 1) / P;
+    const int b0 = p * per, b1 = min(n_chunks, b0 + per);
+    int local = 0;
     if (e < E) {
-        for (int b = 0; b < n_chunks; ++b) {
-            int32_t *p = counts + static_cast<int64_t>(b) * E + e;
-            const int c = *p;
-            *p = run;
+        int b = b0;
+        for (; b + 8 <= b1; b += 8) {
+            int v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = counts[static_cast<int64_t>(b + u) * E + e];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) local += v[u];
+        }
+        for (; b < b1; ++b) local += counts[static_cast<int64_t>(b) * E + e];
+    }
+    part[tid] = local;
+    __syncthreads();
+    // exclusive prefix over p for this expert (P is small)
+    int run = 0;
+    for (int pp = 0; pp < p; ++pp) run += part[pp * Ep + e];
+    if (e < E) {
+        int b = b0;
+        for (; b + 8 <= b1; b += 8) {
+            int v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = counts[static_cast<int64_t>(b + u) * E + e];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                counts[static_cast<int64_t>(b + u) * E + e] = run;
+                run += v[u];
+            }
+        }
+        for (; b < b1; ++b) {
+            const int c = counts[static_cast<int64_t>(b) * E + e];
+            counts[static_cast<int64_t>(b) * E + e] = run;
             run += c;
         }
-        load[e] = run;
+        if (p == P - 1) load[e] = run;
     }
-    sums[e] = e < E ? run : 0;
     __syncthreads();
-    // inclusive Hillis-Steele scan over blockDim.x entries
-    for (int o = 1; o < blockDim.x; o <<= 1) {
-        const int v = e >= o ? sums[e - o] : 0;
+    // exclusive scan of the expert totals into offsets (totals = last pass's run)
+    if (tid < Ep) sums[tid] = 0;
+    __syncthreads();
+    if (p == P - 1 && e < E) sums[e] = run;
+    __syncthreads();
+    for (int o = 1; o < Ep; o <<= 1) {
+        const int v = (tid < Ep && tid >= o) ? sums[tid - o] : 0;
         __syncthreads();
-        sums[e] += v;
+        if (tid < Ep) sums[tid] += v;
         __syncthreads();
     }
-    if (e < E) offsets[e + 1] = sums[e];
-    if (e == 0) offsets[0] = 0;
+    if (tid < E) offsets[tid + 1] = sums[tid];
+    if (tid == 0) offsets[0] = 0;
 }
 
 __global__ void perm_place_kernel(const int32_t *__restrict__ idx, const int32_t *__restrict__ counts,
@@ -93,6 +133,7 @@ __global__ void perm_place_kernel(const int32_t *__restrict__ idx, const int32_t
 }
 
 // One CTA per token: H/16 16-byte vectors of codes plus H/128 scales.
+constexpr int GATHER_V = 4;
 __global__ void __launch_bounds__(128) perm_gather_kernel(const uint4 *__restrict__ xq,
                                                           const float *__restrict__ xs,
                                                           const int32_t *__restrict__ row_of,
@@ -104,11 +145,23 @@ __global__ void __launch_bounds__(128) perm_gather_kernel(const uint4 *__restric
     __syncthreads();
     const int nv = H / 16;
     const uint4 *src = xq + static_cast<int64_t>(t) * nv;
-    for (int v = threadIdx.x; v < nv; v += blockDim.x) {
-        const uint4 d = __ldg(src + v);
+    // issue GATHER_V loads per thread before any store, then fan each out to the K rows
+    for (int v0 = threadIdx.x; v0 < nv; v0 += GATHER_V * blockDim.x) {
+        uint4 d[GATHER_V];
+#pragma unroll
+        for (int u = 0; u < GATHER_V; ++u) {
+            const int v = v0 + u * blockDim.x;
+            d[u] = v < nv ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
+        }
         for (int k = 0; k < K; ++k) {
             const int r = rows[k];
-            if (r >= 0) aq[static_cast<int64_t>(r) * nv + v] = d;
+            if (r < 0) continue;
+            uint4 *dst = aq + static_cast<int64_t>(r) * nv;
+#pragma unroll
+            for (int u = 0; u < GATHER_V; ++u) {
+                const int v = v0 + u * blockDim.x;
+                if (v < nv) dst[v] = d[u];
+            }
         }
     }
     const int ns = H / 128;
@@ -157,7 +210,10 @@ MOE_API int moe_permute(const moe_dims *d, const int32_t *topk_idx, const uint8_
     const int thr = threads_for(d->E);
     const size_t smem = static_cast<size_t>(PERM_CHUNK) * d->K * sizeof(int32_t);
     perm_count_kernel<<<n_chunks, thr, smem, st>>>(topk_idx, counts, d->T, d->K, d->E, status);
-    perm_scan_kernel<<<1, thr, 0, st>>>(counts, n_chunks, d->E, expert_load, expert_offsets);
+    {
+        const int P = SCAN_THREADS / thr;      // chunk partitions per expert
+        perm_scan_kernel<<<1, P * thr, 0, st>>>(counts, n_chunks, d->E, P, expert_load, expert_offsets);
+    }
     perm_place_kernel<<<n_chunks, thr, smem, st>>>(topk_idx, counts, expert_offsets, tok_of, row_of, d->T,
                                                   d->K, d->E);
     if (gather && d->H > 0)
@@ -232,7 +288,10 @@ MOE_API int moe_permute_noalloc(const moe_dims *d, const int32_t *topk_idx, cons
     const int thr = threads_for(d->E);
     const size_t smem = static_cast<size_t>(PERM_CHUNK) * d->K * sizeof(int32_t);
     perm_count_kernel<<<n_chunks, thr, smem, st>>>(topk_idx, counts, d->T, d->K, d->E, status);
-    perm_scan_kernel<<<1, thr, 0, st>>>(counts, n_chunks, d->E, expert_load, expert_offsets);
+    {
+        const int P = SCAN_THREADS / thr;      // chunk partitions per expert
+        perm_scan_kernel<<<1, P * thr, 0, st>>>(counts, n_chunks, d->E, P, expert_load, expert_offsets);
+    }
     perm_place_kernel<<<n_chunks, thr, smem, st>>>(topk_idx, counts, expert_offsets, tok_of, row_of, d->T,
                                                   d->K, d->E);
     if (gather && d->H > 0)

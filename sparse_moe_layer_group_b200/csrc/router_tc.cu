@@ -11,7 +11,8 @@
 // fp32: the fp32 dot product, computed as a bf16 GEMM with K = 3H.
 //
 // router_split_kernel  W fp32 [E, H] -> pieces bf16 [3, E, H]
-// router_tc_kernel     one 128 x 256 tile of logits per CTA over one K split:
+// router_tc_kernel     one 128 x 256 tile of logits per CTA over one K split
+//                      (two CTAs per SM, 256 TMEM columns each):
 //                      warp 0 TMA (x tile 128 x 64 bf16, two 128-row W halves),
 //                      warp 1 TMEM (256 columns) + tcgen05.mma kind::f16,
 //                      warps 2-5 read TMEM and store the fp32 partial sums
@@ -28,7 +29,7 @@ using namespace moe::tc;
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BKE = 64;                 // bf16 elements per 128-byte swizzle row
-constexpr int STAGES = 4;
+constexpr int STAGES = 2;               // 2 x 48 KB: two CTAs share an SM
 constexpr uint32_t A_BYTES = BM * 128;
 constexpr uint32_t B_HALF = 128 * 128;
 constexpr uint32_t STAGE_BYTES = A_BYTES + 2 * B_HALF;
@@ -192,12 +193,12 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 
 }  // namespace rtc
 
-// Number of K splits for T tokens and E experts: enough CTAs to cover the SMs,
-// at least 8 K blocks per split.
+// Number of K splits for T tokens and E experts: enough CTAs to fill every SM
+// with two CTAs, at least 8 K blocks per split.
 int router_splits(int T, int E, int H) {
     const int tiles = ((T + rtc::BM - 1) / rtc::BM) * ((E + rtc::BN - 1) / rtc::BN);
     const int kb_total = 3 * (H / rtc::BKE);
-    int s = num_sms() / (tiles > 0 ? tiles : 1);
+    int s = 2 * num_sms() / (tiles > 0 ? tiles : 1);
     if (s > rtc::MAX_SPLIT) s = rtc::MAX_SPLIT;
     if (s > kb_total / 8) s = kb_total / 8;
     return s < 1 ? 1 : s;
