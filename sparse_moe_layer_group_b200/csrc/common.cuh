@@ -61,11 +61,22 @@ __device__ __forceinline__ void amax_step(float v, float &amax, bool &finite) {
     amax = fmaxf(amax, fabsf(v));
 }
 
-// SwiGLU of one (gate, up) pair in fp32, every operation rounded as written:
-// silu(g) = g / (1 + exp(-g)), act = silu(g) * u.
+// SwiGLU activation silu(g) * u = g / (1 + exp(-g)) * u in fp32, with the
+// hardware exp2 approximation (__expf) and approximate division (__fdividef):
+// a few fp32 ulps from the exact value wherever the result is large enough to
+// set a tile's scale (the error of __expf grows with |g| only where exp(-g)
+// dominates the denominator, i.e. where the activation is near zero).
 __device__ __forceinline__ float swiglu_act(float g, float u) {
-    float den = __fadd_rn(1.0f, expf(-g));
-    return __fmul_rn(__fdiv_rn(g, den), u);
+    return __fmul_rn(__fdividef(g, __fadd_rn(1.0f, __expf(-g))), u);
+}
+
+// E4M3 codes of two activation values against one tile scale, given as its
+// correctly rounded reciprocal (the requantisation of the SwiGLU output:
+// fp32(v * (1/s)) differs from fp32(v / s) by at most one ulp, below the error
+// the activation already carries).  Low byte = a.
+__device__ __forceinline__ uint32_t e4m3x2_rcp(float a, float b, float inv) {
+    return static_cast<uint32_t>(
+        __nv_cvt_float2_to_fp8x2(make_float2(__fmul_rn(a, inv), __fmul_rn(b, inv)), __NV_SATFINITE, __NV_E4M3));
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

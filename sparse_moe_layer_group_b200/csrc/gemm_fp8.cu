@@ -54,16 +54,38 @@ constexpr int EPI_THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAX_G = 4096;
 constexpr int LAUNCH_REGS = 168;   // 384 threads x 168 = 128 x 40 + 256 x 232
+constexpr int EPI_ROW_PITCH = 80;  // 64 data bytes + 16 pad: 16-byte staging stores without bank conflicts
+constexpr uint32_t EPI_STAGE_BYTES = 32 * EPI_ROW_PITCH;
+
+// 64 bytes per thread (the thread's row of the warp's 32 consecutive rows) to
+// dst + row * pitch, through the warp's shared staging buffer, so that every
+// global store instruction writes 8 rows x 64 contiguous bytes rather than
+// 32 rows x 16 bytes.  Rows >= nvalid are not written.  Warp-collective.
+__device__ __forceinline__ void warp_store_rows64(uint8_t *stg, const uint4 (&v)[4], uint8_t *dst, int64_t pitch,
+                                                  int nvalid, int lane) {
+    uint4 *mine = reinterpret_cast<uint4 *>(stg + lane * EPI_ROW_PITCH);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mine[i] = v[i];
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = 8 * i + (lane >> 2), seg = lane & 3;
+        const uint4 w = *reinterpret_cast<const uint4 *>(stg + r * EPI_ROW_PITCH + seg * 16);
+        if (r < nvalid) *reinterpret_cast<uint4 *>(dst + r * pitch + seg * 16) = w;
+    }
+    __syncwarp();
+}
 
 template <bool PAIR>
 struct Cfg {
     static constexpr int TM = PAIR ? 256 : 128;                     // rows per tile (whole pair)
-    static constexpr int STAGES = PAIR ? 6 : 3;     // 3 x 48 KB: a fourth stage measured no faster
+    static constexpr int STAGES = PAIR ? 5 : 3;     // 3 x 48 KB: a fourth stage measured no faster
     static constexpr uint32_t STAGE_BYTES = PAIR ? A_BYTES + B_HALF : A_BYTES + 2 * B_HALF;
     static constexpr uint32_t OFF_BARS = STAGES * STAGE_BYTES;
     static constexpr uint32_t OFF_MISC = OFF_BARS + 256;             // tmem holder, abort, bad
     static constexpr uint32_t OFF_RED = OFF_MISC + 32;               // [2 parity][2 half][128] fp32
-    static constexpr uint32_t OFF_MSTART = OFF_RED + 2 * 2 * 128 * 4;  // int32 [MAX_G + 1]
+    static constexpr uint32_t OFF_EPI = OFF_RED + 2 * 2 * 128 * 4;   // per epilogue warp: store staging
+    static constexpr uint32_t OFF_MSTART = OFF_EPI + 8 * EPI_STAGE_BYTES;  // int32 [MAX_G + 1]
     static constexpr uint32_t SMEM_BYTES = OFF_MSTART + (MAX_G + 1) * 4 + 1024;
     // instruction descriptor: D fp32, A/B e4m3, K-major both, N = 256, M = 128 or 256
     static constexpr uint32_t IDESC = (1u << 4) | (static_cast<uint32_t>(BN >> 3) << 17) |
@@ -202,55 +224,61 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         asm volatile("setmaxnreg.dec.sync.aligned.u32 40;" ::: "memory");
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            int issued = 0;
-            bool ok = true;
-            for (int t = unit; ok && t < num_tiles; t += n_units) {
-                const Tile tl = decode_tile(t, mstart, G, NT, TM, offs);
-                const int r0 = swiglu ? 128 * tl.nt : BN * tl.nt;            // B rows of columns 0..127
-                const int r1 = swiglu ? I + 128 * tl.nt : BN * tl.nt + 128;  // B rows of columns 128..255
-                const int arow = tl.m0 + 128 * static_cast<int>(rank);
-                for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, status)) { ok = false; break; }
-                    const uint32_t sa = sbase + stage * STAGE_BYTES;
-                    if constexpr (PAIR) {
-                        const uint32_t fb = lead_bar0 + 8u * stage;
-                        if (leader) mbar_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
-                        tma_load_2d_pair(sa, &tmA, kb * BK, arow, fb);
-                        tma_load_3d_pair(sa + A_BYTES, &tmB, kb * BK, leader ? r0 : r1, tl.g, fb);
-                    } else {
-                        mbar_expect_tx(full_bar(stage), STAGE_BYTES);
-                        tma_load_2d(sa, &tmA, kb * BK, arow, full_bar(stage));
-                        tma_load_3d(sa + A_BYTES, &tmB, kb * BK, r0, tl.g, full_bar(stage));
-                        tma_load_3d(sa + A_BYTES + B_HALF, &tmB, kb * BK, r1, tl.g, full_bar(stage));
-                    }
-                    ++issued;
-                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        // (the whole warp runs the loop; lane 0 issues)
+        const uint32_t one = lane == 0 ? 1u : 0u;
+        int stage = 0;
+        uint32_t phase = 0;
+        int issued = 0;
+        bool ok = true;
+        for (int t = unit; ok && t < num_tiles; t += n_units) {
+            const Tile tl = decode_tile(t, mstart, G, NT, TM, offs);
+            const int r0 = swiglu ? 128 * tl.nt : BN * tl.nt;            // B rows of columns 0..127
+            const int r1 = swiglu ? I + 128 * tl.nt : BN * tl.nt + 128;  // B rows of columns 128..255
+            const int arow = tl.m0 + 128 * static_cast<int>(rank);
+            for (int kb = 0; kb < KB; ++kb) {
+                ok = __all_sync(0xffffffffu, mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, status));
+                if (!ok) break;
+                const uint32_t sa = sbase + stage * STAGE_BYTES;
+                if constexpr (PAIR) {
+                    const uint32_t fb = lead_bar0 + 8u * stage;
+                    mbar_expect_tx_if(full_bar(stage), 2 * STAGE_BYTES, leader ? one : 0u);
+                    tma_load_2d_pair(sa, &tmA, kb * BK, arow, fb, one);
+                    tma_load_3d_pair(sa + A_BYTES, &tmB, kb * BK, leader ? r0 : r1, tl.g, fb, one);
+                } else {
+                    mbar_expect_tx_if(full_bar(stage), STAGE_BYTES, one);
+                    tma_load_2d(sa, &tmA, kb * BK, arow, full_bar(stage), one);
+                    tma_load_3d(sa + A_BYTES, &tmB, kb * BK, r0, tl.g, full_bar(stage), one);
+                    tma_load_3d(sa + A_BYTES + B_HALF, &tmB, kb * BK, r1, tl.g, full_bar(stage), one);
                 }
+                __syncwarp();
+                ++issued;
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
-            // no TMA write may land after the CTAs exit: wait for the last loads
-            // (in a pair the leader's full barriers count both CTAs' bytes)
-            if (leader) {
-                const int tail = issued < STAGES ? issued : STAGES;
-                for (int i = 0; i < tail; ++i) {
-                    if (stage == 0) { stage = STAGES - 1; phase ^= 1u; } else { --stage; }
-                    mbar_wait(full_bar(stage), phase, abort_flag, status, true);
-                }
+        }
+        // no TMA write may land after the CTAs exit: wait for the last loads
+        // (in a pair the leader's full barriers count both CTAs' bytes)
+        if (leader && lane == 0) {
+            const int tail = issued < STAGES ? issued : STAGES;
+            for (int i = 0; i < tail; ++i) {
+                if (stage == 0) { stage = STAGES - 1; phase ^= 1u; } else { --stage; }
+                mbar_wait(full_bar(stage), phase, abort_flag, status, true);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
-        if (lane == 0 && leader) {
+        // (the whole warp runs the loop; lane 0 issues)
+        if (leader) {
+            const uint32_t one = lane == 0 ? 1u : 0u;
             int stage = 0;
             uint32_t phase = 0, kc = 0;
             bool ok = true;
             for (int t = unit; ok && t < num_tiles; t += n_units) {
                 for (int kb = 0; kb < KB; ++kb, ++kc) {
                     const uint32_t buf = kc & 1u, use = kc >> 1;
-                    if (!mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
-                    if (!mbar_wait(full_bar(stage), phase, abort_flag, status)) { ok = false; break; }
+                    ok = __all_sync(0xffffffffu, mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, status));
+                    if (!ok) break;
+                    ok = __all_sync(0xffffffffu, mbar_wait(full_bar(stage), phase, abort_flag, status));
+                    if (!ok) break;
                     tc_fence_after();
                     const uint32_t sa = sbase + stage * STAGE_BYTES;
                     const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sa + A_BYTES);
@@ -258,22 +286,24 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     if constexpr (PAIR) {
 #pragma unroll
                         for (int k = 0; k < BK / 32; ++k)
-                            mma_f8_pair(d, ad + 2u * k, bd + 2u * k, Cf::IDESC, k > 0 ? 1u : 0u);
-                        mma_commit_pair(empty_bar(stage), 0x3);
-                        mma_commit_pair(tfull_bar(buf), 0x3);
+                            mma_f8_pair(d, ad + 2u * k, bd + 2u * k, Cf::IDESC, k > 0 ? 1u : 0u, one);
+                        mma_commit_pair(empty_bar(stage), 0x3, one);
+                        mma_commit_pair(tfull_bar(buf), 0x3, one);
                     } else {
 #pragma unroll
                         for (int k = 0; k < BK / 32; ++k)
-                            mma_f8(d, ad + 2u * k, bd + 2u * k, Cf::IDESC, k > 0 ? 1u : 0u);
-                        mma_commit(empty_bar(stage));
-                        mma_commit(tfull_bar(buf));
+                            mma_f8(d, ad + 2u * k, bd + 2u * k, Cf::IDESC, k > 0 ? 1u : 0u, one);
+                        mma_commit(empty_bar(stage), one);
+                        mma_commit(tfull_bar(buf), one);
                     }
+                    __syncwarp();
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
             // every MMA of this CTA (pair) has completed before TMEM is released
-            if constexpr (PAIR) mma_commit_pair(drain_bar, 0x1);
-            else mma_commit(drain_bar);
+            if constexpr (PAIR) mma_commit_pair(drain_bar, 0x1, one);
+            else mma_commit(drain_bar, one);
+            __syncwarp();
             mbar_wait(drain_bar, 0, abort_flag, status, true);
         }
     }
@@ -307,7 +337,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 const float s0 = nb1_ok ? __fmul_rn(a_s, __ldg(sb0 + kb)) : 0.0f;
                 const float s1 = nb1_ok ? __fmul_rn(a_s, __ldg(sb1 + kb)) : 0.0f;
                 const uint32_t buf = kc & 1u, use = kc >> 1;
-                if (!mbar_wait(tfull_bar(buf), use & 1u, abort_flag, status)) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, mbar_wait(tfull_bar(buf), use & 1u, abort_flag, status))) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -334,29 +364,44 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             }
             if (!ok) break;
             const bool store_row = grow < tl.m_end;
+            // this warp's 32 rows start at wrow0; the first nvalid of them belong to the group
+            const int64_t wrow0 = static_cast<int64_t>(tl.m0) + 128 * static_cast<int>(rank) + 32 * q;
+            const int64_t left = static_cast<int64_t>(tl.m_end) - wrow0;
+            const int nvalid = left <= 0 ? 0 : (left >= 32 ? 32 : static_cast<int>(left));
+            uint8_t *stg = smem + Cf::OFF_EPI + (warp - 4) * EPI_STAGE_BYTES;
             if (!swiglu) {
                 const int64_t n0 = static_cast<int64_t>(tl.nt) * BN + 128 * half;
-                if (store_row && n0 < N) {
+                if (n0 < N) {
                     if (epi == MOE_EPI_BF16) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(C) + grow * N + n0);
+                        uint8_t *dst = reinterpret_cast<uint8_t *>(C) + (wrow0 * N + n0) * 2;
 #pragma unroll
-                        for (int v = 0; v < 16; ++v) {
-                            uint4 o;
-                            __nv_bfloat162 p0 = __floats2bfloat162_rn(acc[8 * v + 0], acc[8 * v + 1]);
-                            __nv_bfloat162 p1 = __floats2bfloat162_rn(acc[8 * v + 2], acc[8 * v + 3]);
-                            __nv_bfloat162 p2 = __floats2bfloat162_rn(acc[8 * v + 4], acc[8 * v + 5]);
-                            __nv_bfloat162 p3 = __floats2bfloat162_rn(acc[8 * v + 6], acc[8 * v + 7]);
-                            o.x = *reinterpret_cast<uint32_t *>(&p0);
-                            o.y = *reinterpret_cast<uint32_t *>(&p1);
-                            o.z = *reinterpret_cast<uint32_t *>(&p2);
-                            o.w = *reinterpret_cast<uint32_t *>(&p3);
-                            dst[v] = o;
+                        for (int c = 0; c < 4; ++c) {
+                            uint4 v[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const float *f = acc + 32 * c + 8 * i;
+                                __nv_bfloat162 p0 = __floats2bfloat162_rn(f[0], f[1]);
+                                __nv_bfloat162 p1 = __floats2bfloat162_rn(f[2], f[3]);
+                                __nv_bfloat162 p2 = __floats2bfloat162_rn(f[4], f[5]);
+                                __nv_bfloat162 p3 = __floats2bfloat162_rn(f[6], f[7]);
+                                v[i] = make_uint4(*reinterpret_cast<uint32_t *>(&p0), *reinterpret_cast<uint32_t *>(&p1),
+                                                  *reinterpret_cast<uint32_t *>(&p2), *reinterpret_cast<uint32_t *>(&p3));
+                            }
+                            warp_store_rows64(stg, v, dst + 64 * c, 2 * static_cast<int64_t>(N), nvalid, lane);
                         }
                     } else {
-                        float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(C) + grow * N + n0);
+                        uint8_t *dst = reinterpret_cast<uint8_t *>(C) + (wrow0 * N + n0) * 4;
 #pragma unroll
-                        for (int v = 0; v < 32; ++v)
-                            dst[v] = make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+                        for (int c = 0; c < 8; ++c) {
+                            uint4 v[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const float *f = acc + 16 * c + 4 * i;
+                                v[i] = make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                                                  __float_as_uint(f[3]));
+                            }
+                            warp_store_rows64(stg, v, dst + 64 * c, 4 * static_cast<int64_t>(N), nvalid, lane);
+                        }
                     }
                 }
             } else {
@@ -374,31 +419,28 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 rp[half * 128 + row] = fin ? amax : __int_as_float(0x7fc00000);
                 mbar_arrive(xchg_bar(p));
                 uint32_t &xph = p ? xphase1 : xphase0;
-                if (!mbar_wait(xchg_bar(p), xph, abort_flag, status)) { ok = false; break; }
+                // warp-uniform outcome: the staged store below is warp-collective
+                if (!__all_sync(0xffffffffu, mbar_wait(xchg_bar(p), xph, abort_flag, status))) { ok = false; break; }
                 xph ^= 1u;
                 const float mine = rp[half * 128 + row], other = rp[(half ^ 1) * 128 + row];
                 const bool finite = !isnan(mine) && !isnan(other);
                 const float sc = tile_scale(fmaxf(mine, other), finite);
-                if (store_row) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(C) + grow * I +
-                                                           128 * tl.nt + 64 * half);
+                const float inv = __frcp_rn(sc);
+                uint4 v[4];
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int j = 16 * v + 4 * u;
-                            w[u] = static_cast<uint32_t>(quant_code(acc[j], sc, finite)) |
-                                   static_cast<uint32_t>(quant_code(acc[j + 1], sc, finite)) << 8 |
-                                   static_cast<uint32_t>(quant_code(acc[j + 2], sc, finite)) << 16 |
-                                   static_cast<uint32_t>(quant_code(acc[j + 3], sc, finite)) << 24;
-                        }
-                        dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
-                    }
-                    if (half == 0) {
-                        sC[grow * (I / 128) + tl.nt] = sc;
-                        if (!finite) set_flag(status, MOE_FLAG_NONFINITE);
-                    }
+                for (int i = 0; i < 4; ++i) {
+                    const float *f = acc + 16 * i;
+                    v[i] = finite ? make_uint4(e4m3x2_rcp(f[0], f[1], inv) | e4m3x2_rcp(f[2], f[3], inv) << 16,
+                                               e4m3x2_rcp(f[4], f[5], inv) | e4m3x2_rcp(f[6], f[7], inv) << 16,
+                                               e4m3x2_rcp(f[8], f[9], inv) | e4m3x2_rcp(f[10], f[11], inv) << 16,
+                                               e4m3x2_rcp(f[12], f[13], inv) | e4m3x2_rcp(f[14], f[15], inv) << 16)
+                                  : make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+                }
+                warp_store_rows64(stg, v, reinterpret_cast<uint8_t *>(C) + wrow0 * I + 128 * tl.nt + 64 * half,
+                                  static_cast<int64_t>(I), nvalid, lane);
+                if (store_row && half == 0) {
+                    sC[grow * (I / 128) + tl.nt] = sc;
+                    if (!finite) set_flag(status, MOE_FLAG_NONFINITE);
                 }
             }
         }

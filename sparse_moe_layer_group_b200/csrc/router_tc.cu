@@ -109,21 +109,24 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     const uint32_t tmem = *tmem_holder;
 
     if (warp == 0) {
+        // TMA producer: the whole warp runs the loop, lane 0 issues
+        const uint32_t one = lane == 0 ? 1u : 0u;
+        int stage = 0;
+        uint32_t phase = 0;
+        int issued = 0;
+        for (int kb = kb_begin; kb < kb_end; ++kb) {
+            if (!__all_sync(0xffffffffu, mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, status))) break;
+            const int piece = kb / kb_h, k0 = (kb % kb_h) * BKE;
+            const uint32_t sa = sbase + stage * STAGE_BYTES;
+            mbar_expect_tx_if(full_bar(stage), STAGE_BYTES, one);
+            tma_load_2d(sa, &tmX, k0, m0, full_bar(stage), one);
+            tma_load_3d(sa + A_BYTES, &tmW, k0, n0, piece, full_bar(stage), one);
+            tma_load_3d(sa + A_BYTES + B_HALF, &tmW, k0, n0 + 128, piece, full_bar(stage), one);
+            __syncwarp();
+            ++issued;
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            int issued = 0;
-            for (int kb = kb_begin; kb < kb_end; ++kb) {
-                if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, status)) break;
-                const int piece = kb / kb_h, k0 = (kb % kb_h) * BKE;
-                const uint32_t sa = sbase + stage * STAGE_BYTES;
-                mbar_expect_tx(full_bar(stage), STAGE_BYTES);
-                tma_load_2d(sa, &tmX, k0, m0, full_bar(stage));
-                tma_load_3d(sa + A_BYTES, &tmW, k0, n0, piece, full_bar(stage));
-                tma_load_3d(sa + A_BYTES + B_HALF, &tmW, k0, n0 + 128, piece, full_bar(stage));
-                ++issued;
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-            }
             const int tail = issued < STAGES ? issued : STAGES;
             for (int i = 0; i < tail; ++i) {
                 if (stage == 0) { stage = STAGES - 1; phase ^= 1u; } else { --stage; }
@@ -131,25 +134,27 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int i = 0; i < n_kb; ++i) {
-                if (!mbar_wait(full_bar(stage), phase, abort_flag, status)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t sa = sbase + stage * STAGE_BYTES;
-                const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sa + A_BYTES);
+        // MMA issuer: the whole warp runs the loop, lane 0 issues
+        const uint32_t one = lane == 0 ? 1u : 0u;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int i = 0; i < n_kb; ++i) {
+            if (!__all_sync(0xffffffffu, mbar_wait(full_bar(stage), phase, abort_flag, status))) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sa = sbase + stage * STAGE_BYTES;
+            const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sa + A_BYTES);
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_f16(tmem, ad + 2u * k, bd + 2u * k, IDESC, (i > 0 || k > 0) ? 1u : 0u);
-                mma_commit(empty_bar(stage));
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-            }
-            // tfull also serves as the drain: it fires once every MMA issued above is done
-            mma_commit(tfull_bar);
-            if (!ok) mbar_wait(tfull_bar, 0, abort_flag, status, true);
+            for (int k = 0; k < 4; ++k)
+                mma_f16(tmem, ad + 2u * k, bd + 2u * k, IDESC, (i > 0 || k > 0) ? 1u : 0u, one);
+            mma_commit(empty_bar(stage), one);
+            __syncwarp();
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
+        // tfull also serves as the drain: it fires once every MMA issued above is done
+        mma_commit(tfull_bar, one);
+        __syncwarp();
+        if (!ok && lane == 0) mbar_wait(tfull_bar, 0, abort_flag, status, true);
     } else {
         // epilogue: warps 2..5 cover TMEM lane quarters 2, 3, 0, 1
         const int q = warp & 3;

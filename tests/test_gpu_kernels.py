@@ -241,8 +241,10 @@ def test_swiglu_requant_stand_alone(lib):
     torch.cuda.synchronize()
     rq, rs, act = oracle.swiglu_requant(gu.numpy())
     gq, gs = np_(q), np_(s)
-    # scales: fp32 act values differ from the float64 ones by a few ulps
-    assert np.max(np.abs(gs - rs) / rs) < 4 * 2 ** -23
+    # scales: the kernel's act uses __expf (documented error 2 + floor(1.173|x|) ulp)
+    # and __fdividef (2 ulp); for |gate| <= 15 (5 sigma here) that is < 24 ulp on
+    # exp(-g) and, through the denominator, on act, plus roundings: 2^-18 relative
+    assert np.max(np.abs(gs - rs) / rs) < 2.0 ** -18
     same = gq == rq
     assert same.mean() > 0.999
     deq_g = oracle.dequant_1x128(gq, gs)
