@@ -53,6 +53,7 @@ constexpr int THREADS = 384;
 constexpr int EPI_THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAX_G = 4096;
+constexpr uint32_t SMEM_LIMIT = 227 * 1024;   // dynamic shared memory per CTA on sm_100
 constexpr int LAUNCH_REGS = 168;   // 384 threads x 168 = 128 x 40 + 256 x 232
 constexpr int EPI_ROW_PITCH = 80;  // 64 data bytes + 16 pad: 16-byte staging stores without bank conflicts
 constexpr uint32_t EPI_STAGE_BYTES = 32 * EPI_ROW_PITCH;
@@ -85,8 +86,11 @@ struct Cfg {
     static constexpr uint32_t OFF_MISC = OFF_BARS + 256;             // tmem holder, abort, bad
     static constexpr uint32_t OFF_RED = OFF_MISC + 32;               // [2 parity][2 half][128] fp32
     static constexpr uint32_t OFF_EPI = OFF_RED + 2 * 2 * 128 * 4;   // per epilogue warp: store staging
-    static constexpr uint32_t OFF_MSTART = OFF_EPI + 8 * EPI_STAGE_BYTES;  // int32 [MAX_G + 1]
+    static constexpr uint32_t OFF_MSTART = OFF_EPI + 8 * EPI_STAGE_BYTES;  // int32 [G + 1]
+    // launched with smem_bytes(G); the attribute is set once for MAX_G
     static constexpr uint32_t SMEM_BYTES = OFF_MSTART + (MAX_G + 1) * 4 + 1024;
+    static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory layout exceeds the per-CTA limit");
+    static constexpr uint32_t smem_bytes(int G) { return OFF_MSTART + static_cast<uint32_t>(G + 1) * 4u + 1024u; }
     // instruction descriptor: D fp32, A/B e4m3, K-major both, N = 256, M = 128 or 256
     static constexpr uint32_t IDESC = (1u << 4) | (static_cast<uint32_t>(BN >> 3) << 17) |
                                       (static_cast<uint32_t>(TM >> 4) << 24);
@@ -332,10 +336,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             float acc[128];
 #pragma unroll
             for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+            // the three scales of K block kb + 1 are loaded while block kb is promoted
+            float na = row_ok ? __ldg(sa_row) : 0.0f;
+            float nb0v = nb1_ok ? __ldg(sb0) : 0.0f, nb1v = nb1_ok ? __ldg(sb1) : 0.0f;
             for (int kb = 0; kb < KB; ++kb, ++kc) {
-                const float a_s = row_ok ? __ldg(sa_row + kb) : 0.0f;
-                const float s0 = nb1_ok ? __fmul_rn(a_s, __ldg(sb0 + kb)) : 0.0f;
-                const float s1 = nb1_ok ? __fmul_rn(a_s, __ldg(sb1 + kb)) : 0.0f;
+                const float s0 = __fmul_rn(na, nb0v);
+                const float s1 = __fmul_rn(na, nb1v);
+                if (kb + 1 < KB) {
+                    na = row_ok ? __ldg(sa_row + kb + 1) : 0.0f;
+                    nb0v = nb1_ok ? __ldg(sb0 + kb + 1) : 0.0f;
+                    nb1v = nb1_ok ? __ldg(sb1 + kb + 1) : 0.0f;
+                }
                 const uint32_t buf = kc & 1u, use = kc >> 1;
                 if (!__all_sync(0xffffffffu, mbar_wait(tfull_bar(buf), use & 1u, abort_flag, status))) { ok = false; break; }
                 tc_fence_after();
@@ -560,14 +571,14 @@ MOE_API int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets
     cudaStream_t st = as_stream(stream);
     const int n = static_cast<int>(N), k = static_cast<int>(K);
     if (single) {
-        grouped_gemm_kernel<false><<<num_sms(), THREADS, Cfg<false>::SMEM_BYTES, st>>>(
+        grouped_gemm_kernel<false><<<num_sms(), THREADS, Cfg<false>::smem_bytes(G), st>>>(
             tmA, tmB, group_offsets, G, m_capacity, n, k, sA, sB, epilogue, C, sC, status);
         return launch_status();
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pair_clusters(st)), 1, 1);
     cfg.blockDim = dim3(THREADS, 1, 1);
-    cfg.dynamicSmemBytes = Cfg<true>::SMEM_BYTES;
+    cfg.dynamicSmemBytes = Cfg<true>::smem_bytes(G);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
