@@ -21,6 +21,7 @@ bounded sample of the same workload, scaled to tokens/s).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -156,6 +157,32 @@ def build_layer(shape: synth.MoEShape, T: int):
     return layer
 
 
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "grouped_gemm_w13_dsv3_traffic.txt")
+GEMM_SOURCES = ("include/moe_b200.h", "sparse_moe_layer_group_b200/csrc/common.cuh",
+                "sparse_moe_layer_group_b200/csrc/tc_util.cuh", "sparse_moe_layer_group_b200/csrc/gemm_fp8.cu")
+
+
+def recorded_w13_traffic(algorithmic_bytes: int):
+    """DRAM bytes (read + write) of one W13 launch from the committed ncu record,
+    or None when the kernel's sources changed since the record was taken or the
+    record is for another workload (different algorithmic bytes)."""
+    try:
+        with open(TRAFFIC_RECORD) as f:
+            lines = f.read().splitlines()
+        h = hashlib.sha256()
+        for p in GEMM_SOURCES:
+            with open(os.path.join(ROOT, p), "rb") as f:
+                h.update(f.read())
+    except OSError:
+        return None
+    rec = dict(l.split(": ", 1) for l in lines if l and not l.startswith("#") and ": " in l)
+    if rec.get("kernel_sources_sha256") != h.hexdigest():
+        return None
+    if int(rec.get("algorithmic_bytes_per_launch", -1)) != algorithmic_bytes:
+        return None
+    return int(rec["traffic_bytes_per_launch"])
+
+
 def gemm1_bytes(layer, touched: int) -> int:
     """Algorithmic HBM bytes of the W13 grouped GEMM launch: W13 of the touched
     routed experts and of the shared expert, the T*K + T A rows (codes +
@@ -272,7 +299,8 @@ def run_gpu(args, rank, world, local):
         "roofline": {
             "kernel": "grouped_gemm_kernel (W13 of 256 routed + 1 shared expert, SwiGLU+requant epilogue)",
             "bound": "hbm", "achieved": round(g1_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-            "frac": round(g1_gbs / pk["hbm_gbs"], 3), "traffic": None, "peak_kind": pk_kind,
+            "frac": round(g1_gbs / pk["hbm_gbs"], 3), "traffic": recorded_w13_traffic(g1_bytes),
+            "traffic_unit": "bytes per launch", "peak_kind": pk_kind,
             "launch_ms": round(g1_ms, 4), "algorithmic_bytes": g1_bytes, "touched_experts": touched,
             "tensor_tflops": round(g1_tflops, 1), "tensor_frac_of_fp8": round(g1_tflops / fp8_peak, 3),
         },

@@ -1,0 +1,29 @@
+"""Host logic of bench.py that needs no GPU: the ncu traffic record is used only
+while the GEMM kernel's sources are the ones it was taken with."""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_traffic_record_matches_current_sources():
+    rec = dict(l.split(": ", 1) for l in open(bench.TRAFFIC_RECORD).read().splitlines()
+               if l and not l.startswith("#") and ": " in l)
+    alg = int(rec["algorithmic_bytes_per_launch"])
+    got = bench.recorded_w13_traffic(alg)
+    # either the record is current (and then it is what the file says) or stale (None)
+    assert got is None or got == int(rec["traffic_bytes_per_launch"])
+    assert bench.recorded_w13_traffic(alg + 1) is None
+
+
+def test_traffic_record_is_dropped_when_a_source_changes(tmp_path, monkeypatch):
+    changed = tmp_path / "gemm_fp8.cu"
+    with open(os.path.join(ROOT, bench.GEMM_SOURCES[-1]), "rb") as f:
+        changed.write_bytes(f.read() + b"\n// edited\n")
+    monkeypatch.setattr(bench, "GEMM_SOURCES", bench.GEMM_SOURCES[:-1] + (str(changed),))
+    rec = dict(l.split(": ", 1) for l in open(bench.TRAFFIC_RECORD).read().splitlines()
+               if l and not l.startswith("#") and ": " in l)
+    assert bench.recorded_w13_traffic(int(rec["algorithmic_bytes_per_launch"])) is None
