@@ -55,14 +55,39 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) route_select_kernel(
     float *srow = sh + wid * E;
     if (partial) {
         const int64_t plane = static_cast<int64_t>(T) * E;
-        for (int e = lane; e < E; e += 32) {
-            const float *p = partial + static_cast<int64_t>(t) * E + e;
-            float l = p[0];
-            for (int q = 1; q < n_split; ++q) l = __fadd_rn(l, p[q * plane]);
-            if (offset) l = __fadd_rn(l, __ldg(offset + e));
-            const float sv = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l)));
-            srow[e] = sv;
-            if (s_out) s_out[static_cast<int64_t>(t) * E + e] = sv;
+        const float *base = partial + static_cast<int64_t>(t) * E;
+        // eight experts per lane at a time: the eight loads of one split are
+        // independent, so a split costs one memory round trip; every logit is
+        // still summed in split order
+        for (int e0 = 0; e0 < E; e0 += 256) {
+            float l[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int e = e0 + lane + 32 * j;
+                l[j] = e < E ? base[e] : 0.0f;
+            }
+#pragma unroll 4
+            for (int q = 1; q < n_split; ++q) {
+                const float *pq = base + q * plane;
+                float v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int e = e0 + lane + 32 * j;
+                    v[j] = e < E ? pq[e] : 0.0f;
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) l[j] = __fadd_rn(l[j], v[j]);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int e = e0 + lane + 32 * j;
+                if (e < E) {
+                    const float lj = offset ? __fadd_rn(l[j], __ldg(offset + e)) : l[j];
+                    const float sv = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-lj)));
+                    srow[e] = sv;
+                    if (s_out) s_out[static_cast<int64_t>(t) * E + e] = sv;
+                }
+            }
         }
     } else {
         for (int e = lane; e < E; e += 32) srow[e] = s_in[static_cast<int64_t>(t) * E + e];
