@@ -121,14 +121,22 @@ class MoELayer:
         self.out_f32 = None
         self.status = torch.zeros(1, **i32)
 
-    def forward(self, x: torch.Tensor, out_f32: bool = False, stream=None, gemm1_events=None) -> torch.Tensor:
-        """x bf16 [T, H] on the device -> out bf16 [T, H] (self.out).
+    def forward(self, x: torch.Tensor, out_f32: bool = False, stream=None, gemm1_events=None,
+                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """x bf16 [T, H] on the device -> out bf16 [T, H] (self.out, or `out` if
+        given: a caller-owned contiguous bf16 [T, H] device tensor, e.g. one of
+        two buffers while the previous result is still being copied out).
 
         gemm1_events, if given, is a (start, end) pair of CUDA events recorded
         around the W13 grouped GEMM on the launching stream."""
         T, H, E, K, I = self.T, self.H, self.E, self.K, self.I
+        if out is None:
+            out = self.out
+        elif (out.dtype != torch.bfloat16 or tuple(out.shape) != (T, H) or not out.is_contiguous()
+              or out.device != self.out.device):
+            raise ValueError("out must be a contiguous bf16 [T, H] tensor on the layer's device")
         if T == 0:
-            return self.out
+            return out
         if out_f32 and self.out_f32 is None:
             self.out_f32 = torch.empty(T, H, dtype=torch.float32, device=self.out.device)
         st = self.status
@@ -147,9 +155,9 @@ class MoELayer:
             gemm1_events[1].record(torch.cuda.current_stream() if stream is None else stream)
         abi.fp8_grouped_gemm_blockscaled(E + 1, self.offsets_all, M, H, I, self.actq, self.acts, qw.w2, qw.s2,
                                          abi.MOE_EPI_BF16, self.yperm, None, st, stream)
-        abi.moe_combine(self.d, self.yperm, self.row_of, self.topk_w, self.ysh, self.out,
+        abi.moe_combine(self.d, self.yperm, self.row_of, self.topk_w, self.ysh, out,
                         self.out_f32 if out_f32 else None, stream)
-        return self.out
+        return out
 
     def bias_update(self, gamma: float, stream=None, bias: Optional[torch.Tensor] = None):
         """b += gamma * sign(T*K/E - load) from this step's expert loads, into

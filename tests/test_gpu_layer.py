@@ -111,3 +111,18 @@ def test_layer_single_token(lib):
                                     shape.n_group, shape.topk_group, shape.K, shape.rho)
     assert np.array_equal(np_(layer.topk_idx), ref["idx"])
     assert normwise(np_(out), ref["out"]) < TOL_NORMWISE
+
+
+def test_layer_caller_owned_output(lib):
+    """forward(out=buf) writes the same bits into the caller's buffer."""
+    shape = synth.TINY
+    layer, master, wr, b = build_layer(lib, shape, device="cpu")
+    x = cuda(synth.activations(shape.T, shape.H, synth.seed_of(shape, synth.X), shape.x_outlier_frac))
+    ref = layer.forward(x).clone()
+    buf = torch.full_like(ref, float("nan"))
+    got = layer.forward(x, out=buf)
+    torch.cuda.synchronize()
+    assert got.data_ptr() == buf.data_ptr()
+    assert torch.equal(buf, ref)
+    with pytest.raises(ValueError):
+        layer.forward(x, out=torch.empty(shape.T, shape.H, dtype=torch.float32, device="cuda"))
