@@ -420,13 +420,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             } else {
                 // act = silu(g) * u on this thread's 64 columns, amax over the full
                 // 128-column tile via the partner warpgroup (same row, other half)
-                float amax = 0.0f;
-                bool fin = true;
+                // eight independent running maxima (max is exact in any order), so
+                // the 64 steps do not form one dependency chain
+                float am[8];
+                bool fn[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) { am[i] = 0.0f; fn[i] = true; }
 #pragma unroll
                 for (int j = 0; j < 64; ++j) {
                     acc[j] = swiglu_act(acc[j], acc[64 + j]);
-                    amax_step(acc[j], amax, fin);
+                    amax_step(acc[j], am[j & 7], fn[j & 7]);
                 }
+                float amax = am[0];
+                bool fin = fn[0];
+#pragma unroll
+                for (int i = 1; i < 8; ++i) { amax = fmaxf(amax, am[i]); fin = fin && fn[i]; }
                 const int p = iter & 1;
                 float *rp = red + p * 256;
                 rp[half * 128 + row] = fin ? amax : __int_as_float(0x7fc00000);
