@@ -55,22 +55,27 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAX_G = 4096;
 constexpr uint32_t SMEM_LIMIT = 227 * 1024;   // dynamic shared memory per CTA on sm_100
 constexpr int LAUNCH_REGS = 168;   // 384 threads x 168 = 128 x 40 + 256 x 232
-constexpr int EPI_ROW_PITCH = 80;  // 64 data bytes + 16 pad: 16-byte staging stores without bank conflicts
+constexpr int EPI_ROW_PITCH = 144;  // 128 data bytes + 16 pad: 16-byte staging stores without bank conflicts
 constexpr uint32_t EPI_STAGE_BYTES = 32 * EPI_ROW_PITCH;
 
-// 64 bytes per thread (the thread's row of the warp's 32 consecutive rows) to
-// dst + row * pitch, through the warp's shared staging buffer, so that every
-// global store instruction writes 8 rows x 64 contiguous bytes rather than
-// 32 rows x 16 bytes.  Rows >= nvalid are not written.  Warp-collective.
-__device__ __forceinline__ void warp_store_rows64(uint8_t *stg, const uint4 (&v)[4], uint8_t *dst, int64_t pitch,
-                                                  int nvalid, int lane) {
+// Row stores through the warp's shared staging buffer: each thread holds bytes of
+// its own row (the warp owns 32 consecutive rows); they are written to shared
+// memory row by row and read back so that consecutive lanes cover one row, so a
+// global store instruction writes whole row segments (4 rows x 128 bytes, or
+// 8 rows x 64 bytes) rather than 32 rows x 16 bytes.  Rows >= nvalid are not
+// written.  Warp-collective.
+template <int NV>   // 16-byte vectors per thread: 8 (128 bytes) or 4 (64 bytes)
+__device__ __forceinline__ void warp_store_rows(uint8_t *stg, const uint4 (&v)[NV], uint8_t *dst, int64_t pitch,
+                                                int nvalid, int lane) {
+    static_assert(NV == 4 || NV == 8, "row chunk of 64 or 128 bytes");
     uint4 *mine = reinterpret_cast<uint4 *>(stg + lane * EPI_ROW_PITCH);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) mine[i] = v[i];
+    for (int i = 0; i < NV; ++i) mine[i] = v[i];
     __syncwarp();
+    constexpr int ROWS_PER_PASS = 32 / NV;   // lanes per row = NV
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int r = 8 * i + (lane >> 2), seg = lane & 3;
+    for (int i = 0; i < NV; ++i) {
+        const int r = ROWS_PER_PASS * i + lane / NV, seg = lane % NV;
         const uint4 w = *reinterpret_cast<const uint4 *>(stg + r * EPI_ROW_PITCH + seg * 16);
         if (r < nvalid) *reinterpret_cast<uint4 *>(dst + r * pitch + seg * 16) = w;
     }
@@ -388,11 +393,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     if (epi == MOE_EPI_BF16) {
                         uint8_t *dst = reinterpret_cast<uint8_t *>(C) + (wrow0 * N + n0) * 2;
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            uint4 v[4];
+                        for (int c = 0; c < 2; ++c) {
+                            uint4 v[8];
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const float *f = acc + 32 * c + 8 * i;
+                            for (int i = 0; i < 8; ++i) {
+                                const float *f = acc + 64 * c + 8 * i;
                                 __nv_bfloat162 p0 = __floats2bfloat162_rn(f[0], f[1]);
                                 __nv_bfloat162 p1 = __floats2bfloat162_rn(f[2], f[3]);
                                 __nv_bfloat162 p2 = __floats2bfloat162_rn(f[4], f[5]);
@@ -400,20 +405,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                                 v[i] = make_uint4(*reinterpret_cast<uint32_t *>(&p0), *reinterpret_cast<uint32_t *>(&p1),
                                                   *reinterpret_cast<uint32_t *>(&p2), *reinterpret_cast<uint32_t *>(&p3));
                             }
-                            warp_store_rows64(stg, v, dst + 64 * c, 2 * static_cast<int64_t>(N), nvalid, lane);
+                            warp_store_rows<8>(stg, v, dst + 128 * c, 2 * static_cast<int64_t>(N), nvalid, lane);
                         }
                     } else {
                         uint8_t *dst = reinterpret_cast<uint8_t *>(C) + (wrow0 * N + n0) * 4;
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            uint4 v[4];
+                        for (int c = 0; c < 4; ++c) {
+                            uint4 v[8];
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const float *f = acc + 16 * c + 4 * i;
+                            for (int i = 0; i < 8; ++i) {
+                                const float *f = acc + 32 * c + 4 * i;
                                 v[i] = make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
                                                   __float_as_uint(f[3]));
                             }
-                            warp_store_rows64(stg, v, dst + 64 * c, 4 * static_cast<int64_t>(N), nvalid, lane);
+                            warp_store_rows<8>(stg, v, dst + 128 * c, 4 * static_cast<int64_t>(N), nvalid, lane);
                         }
                     }
                 }
@@ -457,7 +462,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                                                e4m3x2_rcp(f[12], f[13], inv) | e4m3x2_rcp(f[14], f[15], inv) << 16)
                                   : make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
                 }
-                warp_store_rows64(stg, v, reinterpret_cast<uint8_t *>(C) + wrow0 * I + 128 * tl.nt + 64 * half,
+                warp_store_rows<4>(stg, v, reinterpret_cast<uint8_t *>(C) + wrow0 * I + 128 * tl.nt + 64 * half,
                                   static_cast<int64_t>(I), nvalid, lane);
                 if (store_row && half == 0) {
                     sC[grow * (I / 128) + tl.nt] = sc;
