@@ -47,6 +47,7 @@ GEMM_CASES = [  # sizes, N, K
     (list(range(0, 300, 7)), 768, 512),         # 43 groups, > 148 tiles: persistent loop
     ([128, 128, 256], 256, 128),                # exact tiles, single K block
     ([600, 0, 255, 256, 1], 512, 384),          # several 256-row pair tiles, ragged
+    ([90, 3, 300, 2100], 512, 256),             # large last group: its tiles are interleaved in two chunks
 ]
 
 
@@ -105,7 +106,7 @@ def test_integer_exact_gemm(lib, mode):
 
 
 @pytest.mark.parametrize("sizes,I,K", [([70, 0, 150], 256, 384), ([1], 128, 128), ([300] * 3, 512, 1024),
-                                       ([257, 511, 3, 0, 129], 256, 256)])
+                                       ([50, 1100], 256, 256), ([257, 511, 3, 0, 129], 256, 256)])
 @pytest.mark.parametrize("mode", list(TILE_MODES))
 def test_grouped_gemm_swiglu_requant(lib, sizes, I, K, mode):
     N = 2 * I
