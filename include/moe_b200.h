@@ -195,7 +195,7 @@ size_t moe_permute_noalloc_max_scratch(void);
  *   MOE_EPI_SWIGLU_REQUANT: B rows 0..I-1 are the gate and I..2I-1 the up
  *   projection (N = 2I); act = silu(g) * u in fp32, then the 1x128 rule of
  *   fp8_quant_1x128: C e4m3 [m_capacity, I], sC fp32 [m_capacity, I/128].
- * Limits: K % 128 == 0, N % 128 == 0 (SwiGLU: I % 128 == 0), G <= 4096.    */
+ * Limits: K % 128 == 0, N % 128 == 0 (SwiGLU: I % 128 == 0), G <= 4000.    */
 int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets, int64_t m_capacity,
                                  int64_t N, int64_t K, const uint8_t *A, const float *sA,
                                  const uint8_t *B, const float *sB, int32_t epilogue, void *C,

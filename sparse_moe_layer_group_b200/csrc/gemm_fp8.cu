@@ -52,11 +52,12 @@ constexpr uint32_t B_HALF = 128 * BK;
 constexpr int THREADS = 384;
 constexpr int EPI_THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int MAX_G = 4096;
+constexpr int MAX_G = 4000;
 constexpr uint32_t SMEM_LIMIT = 227 * 1024;   // dynamic shared memory per CTA on sm_100
 constexpr int LAUNCH_REGS = 168;   // 384 threads x 168 = 128 x 40 + 256 x 232
 constexpr int EPI_ROW_PITCH = 144;  // 128 data bytes + 16 pad: 16-byte staging stores without bank conflicts
-constexpr uint32_t EPI_STAGE_BYTES = 32 * EPI_ROW_PITCH;
+constexpr uint32_t EPI_STAGE_BYTES = 8192;   // per epilogue warp: 32 rows x 256 B (TMA-store layout)
+static_assert(32 * EPI_ROW_PITCH <= EPI_STAGE_BYTES, "row-store staging fits the warp's buffer");
 
 // Row stores through the warp's shared staging buffer: each thread holds bytes of
 // its own row (the warp owns 32 consecutive rows); they are written to shared
@@ -85,13 +86,13 @@ __device__ __forceinline__ void warp_store_rows(uint8_t *stg, const uint4 (&v)[N
 template <bool PAIR>
 struct Cfg {
     static constexpr int TM = PAIR ? 256 : 128;                     // rows per tile (whole pair)
-    static constexpr int STAGES = PAIR ? 5 : 3;     // 3 x 48 KB: a fourth stage measured no faster
+    static constexpr int STAGES = PAIR ? 4 : 3;     // 3 x 48 KB: a fourth stage measured no faster
     static constexpr uint32_t STAGE_BYTES = PAIR ? A_BYTES + B_HALF : A_BYTES + 2 * B_HALF;
-    static constexpr uint32_t OFF_BARS = STAGES * STAGE_BYTES;
+    static constexpr uint32_t OFF_EPI = STAGES * STAGE_BYTES;        // per epilogue warp: store staging (1 KB aligned)
+    static constexpr uint32_t OFF_BARS = OFF_EPI + 8 * EPI_STAGE_BYTES;
     static constexpr uint32_t OFF_MISC = OFF_BARS + 256;             // tmem holder, abort, bad
     static constexpr uint32_t OFF_RED = OFF_MISC + 32;               // [2 parity][2 half][128] fp32
-    static constexpr uint32_t OFF_EPI = OFF_RED + 2 * 2 * 128 * 4;   // per epilogue warp: store staging
-    static constexpr uint32_t OFF_MSTART = OFF_EPI + 8 * EPI_STAGE_BYTES;  // int32 [G + 1]
+    static constexpr uint32_t OFF_MSTART = OFF_RED + 2 * 2 * 128 * 4;  // int32 [G + 1]
     // launched with smem_bytes(G) <= SMEM_LIMIT (the attribute is set once to the limit)
     static constexpr uint32_t SMEM_BYTES = SMEM_LIMIT;
     static constexpr int G_LIMIT = static_cast<int>((SMEM_LIMIT - OFF_MSTART - 1024) / 4) - 1;
@@ -153,6 +154,7 @@ __device__ __forceinline__ int remap_tile(int v, int R, int S, int C) {
 template <bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmC,
                     const int32_t *__restrict__ offs, int G, int64_t m_cap, int N, int K,
                     const float *__restrict__ sA, const float *__restrict__ sB, int epi,
                     void *__restrict__ C, float *__restrict__ sC, int32_t *status) {
@@ -224,6 +226,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     } else if (warp == 3 && lane == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmC)) : "memory");
     }
     if (warp == 1) {
         __syncwarp();
@@ -411,6 +414,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const int64_t left = static_cast<int64_t>(tl.m_end) - wrow0;
             const int nvalid = left <= 0 ? 0 : (left >= 32 ? 32 : static_cast<int>(left));
             uint8_t *stg = smem + Cf::OFF_EPI + (warp - 4) * EPI_STAGE_BYTES;
+            const uint32_t stg_s = sbase + Cf::OFF_EPI + (warp - 4) * EPI_STAGE_BYTES;
+            // a warp whose 32 rows all belong to the group stores them with TMA from
+            // a swizzled staging tile; others store row segments themselves.  Either
+            // way the staging buffer is reused only after the previous TMA store of
+            // this warp has read it.
+            const bool full_warp = nvalid == 32;
+            if (lane == 0) bulk_wait_read();
+            __syncwarp();
             if (!swiglu) {
                 const int64_t n0 = static_cast<int64_t>(tl.nt) * BN + 128 * half;
                 if (n0 < N) {
@@ -429,7 +440,22 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                                 v[i] = make_uint4(*reinterpret_cast<uint32_t *>(&p0), *reinterpret_cast<uint32_t *>(&p1),
                                                   *reinterpret_cast<uint32_t *>(&p2), *reinterpret_cast<uint32_t *>(&p3));
                             }
-                            warp_store_rows<8>(stg, v, dst + 128 * c, 2 * static_cast<int64_t>(N), nvalid, lane);
+                            if (full_warp) {
+                                // box c: 32 rows x 128 B, 128-byte swizzle (chunk i of row r at i ^ (r % 8))
+#pragma unroll
+                                for (int i = 0; i < 8; ++i)
+                                    *reinterpret_cast<uint4 *>(stg + c * 4096 + lane * 128 + ((i ^ (lane & 7)) << 4)) = v[i];
+                            } else {
+                                warp_store_rows<8>(stg, v, dst + 128 * c, 2 * static_cast<int64_t>(N), nvalid, lane);
+                            }
+                        }
+                        if (full_warp) {
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            const uint32_t one = lane == 0 ? 1u : 0u;
+                            tma_store_2d(&tmC, stg_s, static_cast<int32_t>(n0), static_cast<int32_t>(wrow0), one);
+                            tma_store_2d(&tmC, stg_s + 4096, static_cast<int32_t>(n0 + 64), static_cast<int32_t>(wrow0), one);
+                            if (lane == 0) bulk_commit();
                         }
                     } else {
                         uint8_t *dst = reinterpret_cast<uint8_t *>(C) + (wrow0 * N + n0) * 4;
@@ -486,14 +512,28 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                                                e4m3x2_rcp(f[12], f[13], inv) | e4m3x2_rcp(f[14], f[15], inv) << 16)
                                   : make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
                 }
-                warp_store_rows<4>(stg, v, reinterpret_cast<uint8_t *>(C) + wrow0 * I + 128 * tl.nt + 64 * half,
-                                  static_cast<int64_t>(I), nvalid, lane);
+                if (full_warp) {
+                    // one box of 32 rows x 64 B, 64-byte swizzle (chunk i of row r at i ^ ((r / 2) % 4))
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        *reinterpret_cast<uint4 *>(stg + lane * 64 + ((i ^ ((lane >> 1) & 3)) << 4)) = v[i];
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    tma_store_2d(&tmC, stg_s, 128 * tl.nt + 64 * half, static_cast<int32_t>(wrow0), lane == 0 ? 1u : 0u);
+                    if (lane == 0) bulk_commit();
+                } else {
+                    warp_store_rows<4>(stg, v, reinterpret_cast<uint8_t *>(C) + wrow0 * I + 128 * tl.nt + 64 * half,
+                                       static_cast<int64_t>(I), nvalid, lane);
+                }
                 if (store_row && half == 0) {
                     sC[grow * (I / 128) + tl.nt] = sc;
                     if (!finite) set_flag(status, MOE_FLAG_NONFINITE);
                 }
             }
         }
+        // this warp's TMA stores are complete before the CTA exits
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -588,7 +628,7 @@ MOE_API int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets
     auto enc = encode_fn();
     if (!enc) return MOE_ERR_CUDA;
 
-    CUtensorMap tmA, tmB;
+    CUtensorMap tmA, tmB, tmC;
     {
         cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(m_capacity)};
         cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
@@ -614,11 +654,29 @@ MOE_API int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return MOE_ERR_CUDA;
     }
+    // output tiles stored by TMA from the epilogue: bf16 rows in boxes of 32 rows x
+    // 64 columns (128-byte swizzle), SwiGLU codes in boxes of 32 rows x 64 columns
+    // (64-byte swizzle); the fp32 epilogue stores directly (tmC unused)
+    if (epilogue == MOE_EPI_F32) {
+        tmC = tmA;
+    } else {
+        const bool codes = epilogue == MOE_EPI_SWIGLU_REQUANT;
+        const int64_t cols = codes ? N / 2 : N;
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(m_capacity)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(codes ? cols : 2 * cols)};
+        cuuint32_t box[2] = {64, 32};
+        cuuint32_t es[2] = {1, 1};
+        if (enc(&tmC, codes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, dims, strides,
+                box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                codes ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MOE_ERR_CUDA;
+    }
     cudaStream_t st = as_stream(stream);
     const int n = static_cast<int>(N), k = static_cast<int>(K);
     if (single) {
         grouped_gemm_kernel<false><<<num_sms(), THREADS, Cfg<false>::smem_bytes(G), st>>>(
-            tmA, tmB, group_offsets, G, m_capacity, n, k, sA, sB, epilogue, C, sC, status);
+            tmA, tmB, tmC, group_offsets, G, m_capacity, n, k, sA, sB, epilogue, C, sC, status);
         return launch_status();
     }
     cudaLaunchConfig_t cfg = {};
@@ -633,7 +691,7 @@ MOE_API int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<true>, tmA, tmB, group_offsets, G, m_capacity, n, k, sA, sB,
+    if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<true>, tmA, tmB, tmC, group_offsets, G, m_capacity, n, k, sA, sB,
                            static_cast<int>(epilogue), C, sC, status) != cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_status();
