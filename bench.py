@@ -385,14 +385,61 @@ def time_oracle_sample(shape: synth.MoEShape, n_experts: int = 2, seed: int = 0)
                        f"expert rows; est. {t_step:.1f} s per step")}
 
 
+def oracle_step_sampler(shape: synth.MoEShape, tok: int = 256, rows: int = 128):
+    """The reference arm's step: the float64 oracle on a bounded slice of one
+    layer step, scaled to the whole step -- router, top-K, permutation and
+    quantisation of `tok` tokens (a different slice each step) and the FFN of
+    one routed expert on `rows` tokens (128 = the mean expert load T*K/E at the
+    layer shape; the slice is repeated when tok < rows), per-token and per-row times
+    scaled to T tokens and T*K + T expert rows.  Inputs and the expert's
+    quantised weights are prepared once, outside the timing."""
+    import oracle
+    T, H, E, K, I = shape.T, shape.H, shape.E, shape.K, shape.I
+    x = synth.activations(T, H, synth.seed_of(shape, synth.X), shape.x_outlier_frac).float().numpy()
+    wr = synth.router_weights(E, H, shape.wr_std, synth.seed_of(shape, synth.WR)).numpy()
+    b = synth.expert_bias(E, shape.bias_range, synth.seed_of(shape, synth.BIAS)).numpy()
+    w13 = synth.expert_weight(2 * I, H, shape.w_std, synth.seed_of(shape, synth.W13, 0)).float().numpy()
+    w2 = synth.expert_weight(H, I, shape.w_std, synth.seed_of(shape, synth.W2, 0)).float().numpy()
+    q13, s13 = oracle.quant_128x128(w13)
+    q2, s2 = oracle.quant_128x128(w2)
+
+    def step(i: int) -> float:
+        lo = (i * tok) % T
+        xs_ = x[lo:lo + tok]
+        t0 = time.perf_counter()
+        s32 = oracle.router_scores(xs_, wr).astype(np.float32)
+        idx, _ = oracle.select_experts(s32, b, shape.n_group, shape.topk_group, K, shape.rho)
+        oracle.permute(idx, E)
+        xq, xsc = oracle.quant_1x128(xs_)
+        t_route = time.perf_counter() - t0
+        sel = np.arange(rows) % len(xs_)
+        t1 = time.perf_counter()
+        oracle.expert_ffn(xq[sel], xsc[sel], q13, s13, q2, s2)
+        t_ffn = time.perf_counter() - t1
+        t_step = t_route * (T / len(xs_)) + t_ffn / rows * (T * K + T)
+        return T / t_step
+
+    return step
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
+    from threadpoolctl import threadpool_info
     shape = synth.DSV3
-    samples = [time_oracle_sample(shape, seed=i) for i in range(max(1, args.steps))]
-    v = statistics.median(s["value"] for s in samples)
-    cb = dict(samples[0])
-    cb["value"] = round(v, 3)
+    tok, rows = 256, 128
+    step = oracle_step_sampler(shape, tok, rows)
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    vals = [step(args.warmup + i) for i in range(max(1, args.steps))]
+    wall = time.perf_counter() - t0
+    v = statistics.median(vals)
+    threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    cb = {"value": round(v, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+          "sample": (f"per step: router+top-K+permute+quant of {tok} of the {shape.T} tokens and the FFN of one "
+                     f"routed expert on {rows} rows, scaled to {shape.T} tokens and {shape.T * shape.K + shape.T} "
+                     f"expert rows; median over {len(vals)} steps ({wall:.1f} s of host time)")}
     return {
         "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(shape.T / v * 1e3, 1),
