@@ -162,6 +162,20 @@ GEMM_SOURCES = ("include/moe_b200.h", "sparse_moe_layer_group_b200/csrc/common.c
                 "sparse_moe_layer_group_b200/csrc/tc_util.cuh", "sparse_moe_layer_group_b200/csrc/gemm_fp8.cu")
 
 
+def gemm_sources_sha256() -> str:
+    """sha256 of the GEMM's sources with comments and blank space removed, so
+    that an edit of comments alone does not mark the traffic record stale."""
+    import re
+    h = hashlib.sha256()
+    for p in GEMM_SOURCES:
+        with open(os.path.join(ROOT, p)) as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update("".join(src.split()).encode())
+    return h.hexdigest()
+
+
 def recorded_w13_traffic(algorithmic_bytes: int):
     """DRAM bytes (read + write) of one W13 launch from the committed ncu record,
     or None when the kernel's sources changed since the record was taken or the
@@ -169,14 +183,11 @@ def recorded_w13_traffic(algorithmic_bytes: int):
     try:
         with open(TRAFFIC_RECORD) as f:
             lines = f.read().splitlines()
-        h = hashlib.sha256()
-        for p in GEMM_SOURCES:
-            with open(os.path.join(ROOT, p), "rb") as f:
-                h.update(f.read())
+        digest = gemm_sources_sha256()
     except OSError:
         return None
     rec = dict(l.split(": ", 1) for l in lines if l and not l.startswith("#") and ": " in l)
-    if rec.get("kernel_sources_sha256") != h.hexdigest():
+    if rec.get("kernel_sources_sha256") != digest:
         return None
     if int(rec.get("algorithmic_bytes_per_launch", -1)) != algorithmic_bytes:
         return None

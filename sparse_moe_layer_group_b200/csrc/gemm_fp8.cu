@@ -26,14 +26,17 @@
 //
 // CTA organisation (persistent, 384 threads):
 //   warp 0        TMA producer
-//   warp 1        TMEM allocator and MMA issuer (one elected lane; the leader CTA
-//                 only in the pair variant)
+//   warp 1        TMEM allocator and MMA issuer (the leader CTA only in the pair
+//                 variant); both role warps run converged, lane 0 issues
 //   warps 2-3     idle (complete warpgroup 0 for setmaxnreg)
 //   warps 4-11    epilogue: warp w reads TMEM lanes 32*(w%4).., the two
-//                 warpgroups split the 256 accumulator columns
+//                 warpgroups split the 256 accumulator columns; at a tile's end
+//                 each warp writes its 32 output rows through its own shared
+//                 staging tile (TMA store when all 32 rows are the group's)
 // The tile list (group-major, then N tile, then M tile so that CTAs working at
-// the same time share weight tiles through L2) is derived on the device from
-// group_offsets, so no host synchronisation is needed.
+// the same time share weight tiles through L2; the last group cut into two
+// chunks, see remap_tile) is derived on the device from group_offsets, so no
+// host synchronisation is needed.
 //
 // No TMA multicast: every CTA loads its own tiles.  Every wait is bounded (2 s);
 // on expiry the CTA raises MOE_FLAG_TIMEOUT, drains its own outstanding TMA loads

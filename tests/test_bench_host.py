@@ -22,8 +22,17 @@ def test_traffic_record_matches_current_sources():
 def test_traffic_record_is_dropped_when_a_source_changes(tmp_path, monkeypatch):
     changed = tmp_path / "gemm_fp8.cu"
     with open(os.path.join(ROOT, bench.GEMM_SOURCES[-1]), "rb") as f:
-        changed.write_bytes(f.read() + b"\n// edited\n")
+        changed.write_bytes(f.read() + b"\nstatic int edited_code;\n")
     monkeypatch.setattr(bench, "GEMM_SOURCES", bench.GEMM_SOURCES[:-1] + (str(changed),))
     rec = dict(l.split(": ", 1) for l in open(bench.TRAFFIC_RECORD).read().splitlines()
                if l and not l.startswith("#") and ": " in l)
     assert bench.recorded_w13_traffic(int(rec["algorithmic_bytes_per_launch"])) is None
+
+
+def test_comment_edits_keep_the_record(tmp_path, monkeypatch):
+    changed = tmp_path / "gemm_fp8.cu"
+    with open(os.path.join(ROOT, bench.GEMM_SOURCES[-1]), "rb") as f:
+        changed.write_bytes(f.read() + b"\n// a comment\n/* and a\n block */\n")
+    before = bench.gemm_sources_sha256()
+    monkeypatch.setattr(bench, "GEMM_SOURCES", bench.GEMM_SOURCES[:-1] + (str(changed),))
+    assert bench.gemm_sources_sha256() == before
