@@ -554,13 +554,19 @@ def main():
     if args.case:
         run_case(args)
         return
-    rank, world, local = dist_setup(args.gpus)
     if args.impl == "reference":
+        # the oracle runs on the host cores of rank 0 alone; other ranks exit at once
+        # (no process group: nothing is exchanged and rank 0 runs for minutes)
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
         rec = run_reference(args, rank, world)
-    else:
-        rec = run_gpu(args, rank, world, local)
-        if rec is not None and world == 1 and not args.no_cpu_baseline:
-            rec["cpu_baseline"] = time_oracle_sample(synth.DSV3)
+        if rec is not None:
+            print(json.dumps(rec), flush=True)
+        return
+    rank, world, local = dist_setup(args.gpus)
+    rec = run_gpu(args, rank, world, local)
+    if rec is not None and world == 1 and not args.no_cpu_baseline:
+        rec["cpu_baseline"] = time_oracle_sample(synth.DSV3)
     if rec is not None:
         print(json.dumps(rec), flush=True)
     if world > 1:

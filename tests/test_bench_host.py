@@ -36,3 +36,14 @@ def test_comment_edits_keep_the_record(tmp_path, monkeypatch):
     before = bench.gemm_sources_sha256()
     monkeypatch.setattr(bench, "GEMM_SOURCES", bench.GEMM_SOURCES[:-1] + (str(changed),))
     assert bench.gemm_sources_sha256() == before
+
+
+def test_reference_step_sampler_and_rank_split():
+    import argparse
+    import math
+    import synth
+    step = bench.oracle_step_sampler(synth.TINY, tok=32, rows=16)
+    v = step(0)
+    assert math.isfinite(v) and v > 0
+    args = argparse.Namespace(steps=1, warmup=0)
+    assert bench.run_reference(args, rank=1, world=2) is None    # only rank 0 works
