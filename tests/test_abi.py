@@ -72,6 +72,10 @@ def test_host_validation_rejects_before_launch():
                                           None) == a.MOE_ERR_INVALID_ARG
     assert L.fp8_grouped_gemm_blockscaled(1, 16, 64, 256, 128, 16, 16, 16, 16, 2, 16, None, None,
                                           None) == a.MOE_ERR_INVALID_ARG
+    # more groups than the kernel's shared-memory group table holds (limit 4000, both tile modes)
+    for mode in (0, a.MOE_GEMM_PAIR_CTA):
+        assert L.fp8_grouped_gemm_blockscaled(4001, 16, 64, 256, 128, 16, 16, 16, 16, mode, 16, None, None,
+                                              None) == a.MOE_ERR_UNSUPPORTED
     # zero-size work is a no-op
     assert L.fp8_grouped_gemm_blockscaled(0, 16, 64, 256, 128, 16, 16, 16, 16, 0, 16, None, None, None) == 0
     assert L.fp8_quant_1x128(16, 0, 128, 16, 16, None, None) == 0
