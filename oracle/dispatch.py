@@ -6,8 +6,8 @@ The pages give the semantics y = sum_j gate_j * ffn_{idx_j}(h) with no token
 ever dropped ([report-walkthrough] section 3.2 pseudocode and section 3.4:
 no capacity factor, every token reaches all K experts) and a dispatch /
 expert MLP / combine split of the forward block ([report-walkthrough]
-section 4.1).  They give no layout.  The layout used (a reading, listed in
-the design doc): rows grouped by expert in ascending expert order, and within an
+section 4.1).  They give no layout.  The layout used (a reading of
+the pages): rows grouped by expert in ascending expert order, and within an
 expert in ascending token order (a stable sort by expert); the x rows are
 quantised first and their codes gathered (1x128 tiles lie inside one token
 row, so quantise-then-gather equals gather-then-quantise bit for bit).

@@ -6,7 +6,7 @@ Test infrastructure only (see the package docstring).
 their own scales and accumulation stays in higher precision.  [infra-answer]:
 the per-tile (1x128) / per-group (128x128) scales are not supported by the
 tensor cores, so the product is formed as partial sums that are promoted.
-Reading (DESIGN.md): for every 128-wide block kb of K,
+Reading: for every 128-wide block kb of K,
     P_kb[m, n] = sum_{k in kb} decode(qa[m, k]) * decode(qb[n, k])
     C[m, n]   += sA[m, kb] * sB[n // 128, kb] * P_kb[m, n].
 P_kb is exact in float64 (products of two E4M3 values have at most 8

@@ -13,7 +13,7 @@ section 3 (input_quant_granularity tile_wise_1x128, weight_quant_granularity
 block_wise_128x128, format e4m3) and [infra-answer] (E4M3 everywhere, per-tile
 1x128 and per-group 128x128): one scale per 1x128 tile of an activation row
 and per 128x128 block of a weight.  The pages do not spell the scale rule
-out; the reading used here (stated in the design doc's readings) is
+out; the reading used here is
     amax  = max |v| over the tile,
     scale = fp32(amax / 448)            (one correctly rounded fp32 division)
     q     = e4m3_rne_satfinite(fp32(v / scale))

@@ -12,7 +12,8 @@ recipe of section 4.3 and [repro-guide] section 3):
   5. out[t] = sum_k w[t,k] y_{t,k} + y_shared[t], stored as bf16.
   6. load = bincount(idx) drives the bias update (separate call).
 The layer input x is the already-normalised hidden state; there is no
-residual add here (a reading).
+residual add here (a reading: the pages place the norm and residual outside
+the MoE FFN).
 """
 from __future__ import annotations
 

@@ -15,7 +15,7 @@ routing ([report-walkthrough] section 3.4): each token is sent to at most M
 nodes, chosen by the sum of the highest affinities of the experts on each
 node; here a "node" is one of n_group equal expert groups, M = topk_group.
 
-Readings where the pages are silent (listed in the design doc):
+Readings where the pages are silent:
 * the group score is the sum of the top min(2, E/n_group) values of s + b in
   the group, added in fp32;
 * ties go to the lower index (groups and experts); output order is

@@ -609,7 +609,8 @@ MOE_API int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets
                                          float *sC, int32_t *status, void *stream) {
     using namespace moe::gg;
     // tile mode: one-SM tiles unless CTA pairs are asked for (measured on B200:
-    // pairs are no faster at the shapes of this layer)
+    // pairs are 25 % slower at 128 tokens per expert, where 256-row tiles are
+    // mostly padding, and about 1 % faster at 1024 tokens per expert)
     const bool single = (epilogue & MOE_GEMM_PAIR_CTA) == 0 || (epilogue & MOE_GEMM_SINGLE_CTA) != 0;
     epilogue &= ~(MOE_GEMM_SINGLE_CTA | MOE_GEMM_PAIR_CTA);
     if (G < 0 || m_capacity < 0 || N < 0 || K < 0) return MOE_ERR_INVALID_ARG;

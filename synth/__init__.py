@@ -63,7 +63,7 @@ class MoEShape:
     seed_base: int = 0
 
 
-# BASELINE-style named workloads (sizes as the pages give them).
+# Named workloads (sizes as the pages give them).
 TINY = MoEShape("tiny", T=64, H=256, E=16, K=4, n_group=4, topk_group=2, I=128,
                 wr_std=0.02, w_std=0.02, bias_range=0.01, seed_base=0)
 DSV3 = MoEShape("dsv3", T=4096, H=7168, E=256, K=8, n_group=8, topk_group=4, I=2048,
