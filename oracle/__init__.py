@@ -51,3 +51,4 @@ __all__ = [
     "gemm_blockscaled", "grouped_gemm_blockscaled", "silu", "swiglu", "swiglu_requant", "expert_ffn",
     "LayerWeights", "quantize_layer_weights", "moe_forward", "moe_forward_tokens",
 ]
+from .backward import quant_128x1, dgrad_blockscaled, wgrad_blockscaled
