@@ -149,3 +149,45 @@ def test_bad_offsets_flagged(lib, mode):
     torch.cuda.synchronize()
     assert int(st.item()) & lib.MOE_FLAG_BAD_OFFSETS
     assert torch.all(C == 3.0)
+
+
+@pytest.mark.parametrize("mode", list(TILE_MODES))
+def test_dgrad_through_the_grouped_gemm(lib, mode):
+    """Backward dgrad dX = dY . W per expert runs on the forward kernel with the
+    weights quantised transposed: 128x128 block codes and scales transpose
+    exactly, so B = W^T [K, N] with contraction over N reproduces the oracle's
+    dgrad (promotion per 128 of N)."""
+    from oracle.backward import dgrad_blockscaled
+    sizes, N, K = [70, 0, 150], 256, 384            # forward Y [M, N] = X [M, K] W^T, W [N, K]
+    G = len(sizes)
+    M = sum(sizes)
+    offs = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    dy = synth.heavy_tailed(M, N, 41)
+    w = synth.normal((G * N, K), 0.02, 42, dtype=torch.bfloat16).reshape(G, N, K)
+    dyq, sdy = oracle.quant_1x128(dy.float().numpy())
+    ref = np.zeros((M, K))
+    wq_ref = []
+    for g in range(G):
+        wq, sw = oracle.quant_128x128(w[g].float().numpy())
+        wq_ref.append((wq, sw))
+        r0, r1 = offs[g], offs[g + 1]
+        if r1 > r0:
+            ref[r0:r1] = dgrad_blockscaled(dyq[r0:r1], sdy[r0:r1], wq, sw)
+    qdy = torch.empty(M, N, dtype=torch.uint8, device="cuda")
+    qsdy = torch.empty(M, N // 128, dtype=torch.float32, device="cuda")
+    lib.fp8_quant_1x128(cuda(dy), qdy, qsdy)
+    wt = cuda(w.transpose(1, 2))                          # [G, K, N]
+    qwt = torch.empty(G, K, N, dtype=torch.uint8, device="cuda")
+    swt = torch.empty(G, K // 128, N // 128, dtype=torch.float32, device="cuda")
+    lib.fp8_quant_128x128(wt, qwt, swt)
+    for g in range(G):                                    # transposed quantisation is exact
+        assert np.array_equal(np_(qwt[g]), wq_ref[g][0].T) and np.array_equal(np_(swt[g]), wq_ref[g][1].T)
+    dx = torch.zeros(M, K, dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lib.fp8_grouped_gemm_blockscaled(G, cuda(torch.from_numpy(offs)), M, K, N, qdy, qsdy, qwt, swt,
+                                     lib.MOE_EPI_F32 | TILE_MODES[mode], dx, None, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    got = np_(dx)
+    assert normwise(got, ref) < TOL_NORMWISE
+    assert np.all(np.abs(got - ref) <= 1e-4 * np.abs(ref) + 1e-5 * np.abs(ref).max())
