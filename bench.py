@@ -138,7 +138,10 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- GPU arm
-def build_layer(shape: synth.MoEShape, T: int):
+def build_layer(shape: synth.MoEShape, T: int, qw=None, offset=None):
+    """The layer of `shape` for T tokens: its router and bias from the shape's
+    seeds; expert weights drawn and quantised here unless `qw` (the resident
+    E4M3 weights of another layer of the same sizes) is given."""
     import sparse_moe_layer_group_b200 as moe
     H, E, I = shape.H, shape.E, shape.I
 
@@ -150,10 +153,12 @@ def build_layer(shape: synth.MoEShape, T: int):
         rows, cols = (2 * I, H) if kind == "w13" else (H, I)
         return synth.expert_weight(rows, cols, shape.w_std, synth.seed_of(shape, tid, max(e, 0)), device="cuda")
 
-    qw = moe.QuantWeights.from_master(master, E, H, I, device="cuda")
+    if qw is None:
+        qw = moe.QuantWeights.from_master(master, E, H, I, device="cuda")
     wr = synth.router_weights(E, H, shape.wr_std, synth.seed_of(shape, synth.WR), device="cuda")
     b = synth.expert_bias(E, shape.bias_range, synth.seed_of(shape, synth.BIAS), device="cuda")
-    layer = moe.MoELayer(T, H, E, shape.K, shape.n_group, shape.topk_group, I, shape.rho, wr, b, qw)
+    layer = moe.MoELayer(T, H, E, shape.K, shape.n_group, shape.topk_group, I, shape.rho, wr, b, qw,
+                         router_offset=offset)
     return layer
 
 
@@ -216,16 +221,16 @@ def run_gpu(args, rank, world, local):
     stream = torch.cuda.current_stream()
     pk, pk_kind = peaks()
 
-    # the dominant kernel's launches are bracketed with events on the same stream
-    g1_events = []
+    # the GEMM launches are bracketed with events on the same stream
+    g_events = []
     b_next = layer.e_bias.clone()
 
     def step(record=False):
         ev = None
         if record:
-            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            g1_events.append(ev)
-        layer.forward(x, gemm1_events=ev)
+            ev = tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
+            g_events.append(ev)
+        layer.forward(x, gemm_events=ev)
         # the bias update runs every step; its result goes to b_next so the
         # workload keeps the configured routing bias b = 0
         layer.bias_update(gamma, bias=b_next)
@@ -249,7 +254,8 @@ def run_gpu(args, rank, world, local):
     ms = t0.elapsed_time(t1)
     ms_max = reduce_max(ms, world)
     status = int(layer.status.item())
-    g1_ms = sum(a.elapsed_time(b) for a, b in g1_events) / len(g1_events)
+    g1_ms = sum(a.elapsed_time(b) for a, b, _ in g_events) / len(g_events)
+    g2_ms = sum(b.elapsed_time(c) for _, b, c in g_events) / len(g_events)
     load = layer.load.cpu().numpy()
     touched = int((load > 0).sum())
     seq_loss, entropy = layer.balance_stats(T, 0.001)     # one 4096-token sequence per step
@@ -347,12 +353,150 @@ def run_gpu(args, rank, world, local):
                 "h2d_bytes_per_step": T * shape.H * 2, "d2h_bytes_per_step": T * shape.H * 2,
                 "how": "MoELayer.forward per step; pinned-host input copied in and output copied back on two "
                        "copy streams overlapping the adjacent steps' compute (double-buffered device input/output)"},
+        "w2_launch_ms": round(g2_ms, 4),
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "device_status": status,
         "balance": balance,
     }
+    if world == 1 and not args.no_workloads:
+        rec["workloads"] = run_workloads(layer.qw, pk, pk_kind)
     return rec
+
+
+# ----------------------------------------------------------------- further workloads
+def _gemm_flops(T: int, K: int, H: int, I: int):
+    rows = T * K + T                   # routed (token, slot) rows + the shared expert's T rows
+    return 2 * rows * 2 * I * H, 2 * rows * H * I
+
+
+def leg_prefill(qw, pk, steps: int = 20) -> dict:
+    """Prefill-scale skewed routing: T = 32768 at the DeepSeek-V3 shape, router
+    logits offset by a Zipf(1.1) ranking (initial max/mean expert load ~20),
+    `steps` consecutive forwards each followed by the bias update (gamma 0.001)
+    that feeds back into the next step's routing; a fresh batch every step."""
+    s = synth.PREFILL
+    T, H, E, K, I = s.T, s.H, s.E, s.K, s.I
+    off = synth.zipf_offset(E, synth.zipf_kappa_default(), synth.seed_of(s, synth.ZIPF), device="cuda")
+    layer = build_layer(s, T, qw=qw, offset=off)
+    xs = [synth.activations(T, H, synth.seed_of(s, synth.X) + 1000 * i, s.x_outlier_frac, device="cuda")
+          for i in range(steps)]
+    b0 = layer.e_bias.clone()
+    layer.forward(xs[0])                       # warm-up, then back to the initial bias
+    layer.e_bias.copy_(b0)
+    hist = torch.empty(steps, E, dtype=torch.int32, device="cuda")
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(steps)]
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        layer.forward(xs[i], gemm_events=ev[i])
+        layer.bias_update(0.001)
+        hist[i].copy_(layer.load, non_blocking=True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    w13 = [a.elapsed_time(b) for a, b, _ in ev]
+    w2 = [b.elapsed_time(c) for _, b, c in ev]
+    f13, f2 = _gemm_flops(T, K, H, I)
+    loads = hist.cpu().numpy().astype(np.float64)
+    ratio = loads.max(axis=1) / loads.mean(axis=1)
+    peak = 2.0 * pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    del xs, layer
+    return {"workload": workload_desc(s) + " + Zipf(1.1) router offset, bias update fed back each step",
+            "steps": steps, "ms_per_step": round(ms, 4), "tokens_per_s": round(T / (ms / 1e3), 1),
+            "w13_ms": round(statistics.mean(w13), 4), "w2_ms": round(statistics.mean(w2), 4),
+            "w13_tflops": round(f13 / statistics.mean(w13) / 1e9, 1),
+            "w2_tflops": round(f2 / statistics.mean(w2) / 1e9, 1),
+            "gemm_tflops": round((f13 + f2) / (statistics.mean(w13) + statistics.mean(w2)) / 1e9, 1),
+            "gemm_frac_of_fp8_peak": round((f13 + f2) / (statistics.mean(w13) + statistics.mean(w2)) / 1e9 / peak, 3),
+            "fp8_peak_tflops": peak, "fp8_peak_kind": "2 x bf16_tflops_sustained (measured)",
+            "max_over_mean_load_first": round(float(ratio[0]), 3),
+            "max_over_mean_load_last": round(float(ratio[-1]), 3)}
+
+
+def leg_decode(qw, pk, steps: int = 50) -> dict:
+    """Decode-sized batch: T = 128 tokens at the DeepSeek-V3 shape, all 257
+    experts' E4M3 weights resident; judged by the HBM bandwidth of the expert
+    weights the step actually touches (every expert with a routed token, plus
+    the shared expert), read by the two grouped GEMMs."""
+    s = synth.DECODE
+    T, H, E, K, I = s.T, s.H, s.E, s.K, s.I
+    layer = build_layer(s, T, qw=qw)
+    x = synth.activations(T, H, synth.seed_of(s, synth.X), s.x_outlier_frac, device="cuda")
+    for _ in range(3):
+        layer.forward(x)
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(steps)]
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        layer.forward(x, gemm_events=ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    gemm_ms = statistics.mean(a.elapsed_time(c) for a, _, c in ev)
+    touched = int((layer.load.cpu().numpy() > 0).sum()) + 1
+    per_expert = 3 * I * H + ((2 * I // 128) * (H // 128) + (H // 128) * (I // 128)) * 4
+    wbytes = touched * per_expert
+    gbs = wbytes / (gemm_ms / 1e3) / 1e9
+    del layer
+    return {"workload": workload_desc(s), "steps": steps, "ms_per_step": round(ms, 4),
+            "tokens_per_s": round(T / (ms / 1e3), 1), "gemm_ms": round(gemm_ms, 4),
+            "touched_experts": touched, "touched_weight_bytes": wbytes,
+            "weight_gbs": round(gbs, 1), "weight_frac_of_hbm": round(gbs / pk["hbm_gbs"], 3),
+            "l2": "no flush: ~11 GB of touched weights per step exceed the 126 MB L2"}
+
+
+def leg_gemm_dense(pk, M: int = 4096, N: int = 18432, K: int = 7168, iters: int = 20) -> dict:
+    """Dense FP8 block-scaled GEMM of the sweep: A [M, K] bf16 N(0,1) with 1 % of
+    the entries x100, quantised 1x128; B [N, K] N(0, 0.02) in 128x128 blocks;
+    C bf16.  Each launch is timed alone after an L2 flush (a 256 MB write)."""
+    import sparse_moe_layer_group_b200 as moe
+    abi = moe.abi
+    a = synth.heavy_tailed(M, K, 71, device="cuda")
+    qa = torch.empty(M, K, dtype=torch.uint8, device="cuda")
+    sa = torch.empty(M, K // 128, dtype=torch.float32, device="cuda")
+    abi.fp8_quant_1x128(a, qa, sa)
+    b = synth.normal((N, K), 0.02, 72, device="cuda", dtype=torch.bfloat16)
+    qb = torch.empty(1, N, K, dtype=torch.uint8, device="cuda")
+    sb = torch.empty(1, N // 128, K // 128, dtype=torch.float32, device="cuda")
+    abi.fp8_quant_128x128(b, qb[0], sb[0])
+    del a, b
+    C = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    offs = torch.tensor([0, M], dtype=torch.int32, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    run = lambda: abi.fp8_grouped_gemm_blockscaled(1, offs, M, N, K, qa, sa, qb, sb, abi.MOE_EPI_BF16, C)
+    for _ in range(3):
+        run()
+    times = []
+    for _ in range(iters):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run()
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    tflops = 2 * M * N * K / (ms / 1e3) / 1e12
+    peak = 2.0 * pk["bf16_tflops"]
+    return {"workload": f"dense FP8 block-scaled GEMM M={M} N={N} K={K}, bf16 out", "launches": iters,
+            "ms": round(ms, 4), "tflops": round(tflops, 1), "frac_of_fp8_peak": round(tflops / peak, 3),
+            "fp8_peak_tflops": peak, "fp8_peak_kind": "2 x bf16_tflops burst (measured)",
+            "l2": "flushed before every launch (256 MB write)"}
+
+
+def run_workloads(qw, pk, pk_kind) -> dict:
+    """The other configurations of the layer, each timed with CUDA events only:
+    prefill with skewed routing, decode, and the dense GEMM sweep's largest
+    compute-bound shape.  The layer legs reuse the resident DeepSeek-V3 expert
+    weights (same sizes); their routers and inputs come from their own seeds."""
+    out = {"prefill_skew": leg_prefill(qw, pk), "decode": leg_decode(qw, pk), "gemm_dense": leg_gemm_dense(pk)}
+    torch.cuda.empty_cache()
+    return out
 
 
 # ----------------------------------------------------------------- CPU oracle arm
@@ -547,6 +691,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the prefill / decode / dense-GEMM legs reported under 'workloads'")
     ap.add_argument("--case", default=None,
                     help="time one kernel alone: gemm1 | gemm1_x256 | gemm1_skew | gemm2 | router")
     ap.add_argument("--gemm-mode", default="auto", choices=["auto", "single", "pair"])

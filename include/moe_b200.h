@@ -132,6 +132,21 @@ int moe_route(const moe_dims *dims, const void *x, const float *w_router, const 
               const float *router_offset, int32_t *topk_idx, float *topk_w, float *scores,
               void *ws, size_t ws_bytes, int32_t *status, void *stream);
 
+/* The router weights split once, for callers that route many batches with the
+ * same W_r: moe_router_split writes the three exact bf16 pieces of W_r
+ * (W_r = P0 + P1 + P2 element by element: P0 = bf16(W_r), P1 = bf16(W_r - P0),
+ * P2 = W_r - P0 - P1, which has at most 8 significant bits), the operand of
+ * moe_route's tensor-core logits; moe_route_pieces is moe_route with those
+ * pieces in place of w_router and gives the same bits.  The pieces stay valid
+ * until W_r changes.
+ *   w_router fp32 [E, H];  w_pieces bf16 [3, E, H] (moe_router_pieces_bytes)
+ *   moe_route_pieces takes the workspace of moe_route (moe_workspace_size). */
+size_t moe_router_pieces_bytes(int32_t E, int32_t H);
+int moe_router_split(const float *w_router, int32_t E, int32_t H, void *w_pieces, void *stream);
+int moe_route_pieces(const moe_dims *dims, const void *x, const void *w_pieces, const float *e_bias,
+                     const float *router_offset, int32_t *topk_idx, float *topk_w, float *scores,
+                     void *ws, size_t ws_bytes, int32_t *status, void *stream);
+
 /* The selection half of moe_route alone, on given affinities s fp32 [T, E]. */
 int moe_route_select(const moe_dims *dims, const float *scores, const float *e_bias,
                      int32_t *topk_idx, float *topk_w, void *stream);

@@ -54,6 +54,9 @@ _SIGS = {
     "fp8_quant_128x128": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P]),
     "moe_route": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "moe_route_select": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P]),
+    "moe_router_pieces_bytes": (_SZ, [_I32, _I32]),
+    "moe_router_split": (ctypes.c_int, [_P, _I32, _I32, _P, _P]),
+    "moe_route_pieces": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "moe_permute": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "moe_permute_noalloc": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_permute_noalloc_max_scratch": (_SZ, []),
@@ -130,6 +133,24 @@ def moe_route(d, x, w_router, e_bias, router_offset, topk_idx, topk_w, scores=No
     _check("moe_route", _lib.moe_route(ctypes.byref(d), _ptr(x), _ptr(w_router), _ptr(e_bias),
                                        _ptr(router_offset), _ptr(topk_idx), _ptr(topk_w), _ptr(scores),
                                        _ptr(ws), ws_bytes, _ptr(status), _stream(stream)))
+
+
+def moe_router_pieces_bytes(E, H) -> int:
+    return int(_lib.moe_router_pieces_bytes(int(E), int(H)))
+
+
+def moe_router_split(w_router, w_pieces, stream=None):
+    E, H = w_router.shape
+    _check("moe_router_split", _lib.moe_router_split(_ptr(w_router), E, H, _ptr(w_pieces), _stream(stream)))
+
+
+def moe_route_pieces(d, x, w_pieces, e_bias, router_offset, topk_idx, topk_w, scores=None, ws=None,
+                     status=None, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("moe_route_pieces", _lib.moe_route_pieces(ctypes.byref(d), _ptr(x), _ptr(w_pieces), _ptr(e_bias),
+                                                     _ptr(router_offset), _ptr(topk_idx), _ptr(topk_w),
+                                                     _ptr(scores), _ptr(ws), ws_bytes, _ptr(status),
+                                                     _stream(stream)))
 
 
 def moe_route_select(d, scores, e_bias, topk_idx, topk_w, stream=None):

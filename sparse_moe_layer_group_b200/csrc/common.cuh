@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/moe_b200.h"
 
 #define MOE_API extern "C" __attribute__((visibility("default")))
@@ -21,15 +23,37 @@ inline int launch_status() {
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+constexpr int MAX_DEVICES = 64;
+
+// The current device, or -1 when it cannot be queried.
+inline int current_device() {
+    int dev = -1;
+    return cudaGetDevice(&dev) == cudaSuccess ? dev : -1;
+}
+
+// Per-device, once-only set-up (kernel attributes, occupancy queries): runs
+// `fn` for the current device the first time and returns its cached result
+// afterwards.  `state` and `mu` belong to one call site; thread-safe.  fn
+// returns a positive value on success; a non-positive result is not cached.
+template <typename F>
+inline int once_per_device(int (&state)[MAX_DEVICES], std::mutex &mu, F fn) {
+    const int dev = current_device();
+    if (dev < 0 || dev >= MAX_DEVICES) return fn();
+    std::lock_guard<std::mutex> lock(mu);
+    if (state[dev] <= 0) state[dev] = fn();
+    return state[dev];
+}
+
+// Number of SMs of the current device (cached per device).
 inline int num_sms() {
-    static int cached = 0;
-    if (cached == 0) {
+    static int state[MAX_DEVICES] = {};
+    static std::mutex mu;
+    return once_per_device(state, mu, []() {
         int dev = 0, n = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        cached = n > 0 ? n : 148;
-    }
-    return cached;
+        return n > 0 ? n : 148;
+    });
 }
 
 __device__ __forceinline__ void set_flag(int32_t *status, int32_t bit) {
@@ -70,13 +94,47 @@ __device__ __forceinline__ float swiglu_act(float g, float u) {
     return __fmul_rn(__fdividef(g, __fadd_rn(1.0f, __expf(-g))), u);
 }
 
-// E4M3 codes of two activation values against one tile scale, given as its
-// correctly rounded reciprocal (the requantisation of the SwiGLU output:
-// fp32(v * (1/s)) differs from fp32(v / s) by at most one ulp, below the error
-// the activation already carries).  Low byte = a.
+// E4M3 codes of fp32(a / s) and fp32(b / s), the correctly rounded quotients
+// of the quantisation rule, for a tile whose scale s has the correctly rounded
+// reciprocal inv = 1/s.  Low byte = a.
+//
+// q = fp32(v * inv) differs from v / s by at most 2^-24 |v/s| (the reciprocal)
+// plus half an ulp (the product), so the correctly rounded quotient lies
+// within three steps of the fp32 grid from q, on q's side of zero.  E4M3
+// rounding is monotone in the magnitude, so when |q| lowered and raised by four
+// grid steps gives the same code, that code is the quotient's; otherwise (a
+// quotient within a few fp32 ulps of an E4M3 rounding boundary, or a reciprocal
+// that overflowed) the quotient is computed by the correctly rounded division.
+__device__ __forceinline__ uint32_t e4m3x2_cvt(float a, float b) {
+    return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
+}
+__device__ __forceinline__ float grid_steps(float q, int n) {   // |q| moved by n fp32 steps, sign kept
+    const uint32_t u = __float_as_uint(q), sgn = u & 0x80000000u;
+    const int m = static_cast<int>(u ^ sgn) + n;   // |q| < 2^31 as a bit pattern
+    return __uint_as_float(sgn | static_cast<uint32_t>(m < 0 ? 0 : m));
+}
+// E4M3 codes of fp32(a * inv) and fp32(b * inv), inv the correctly rounded
+// reciprocal of the tile scale: the fast form of the requantisation, within 1.5
+// fp32 ulps of the quotient before the E4M3 rounding.  Low byte = a.
 __device__ __forceinline__ uint32_t e4m3x2_rcp(float a, float b, float inv) {
-    return static_cast<uint32_t>(
-        __nv_cvt_float2_to_fp8x2(make_float2(__fmul_rn(a, inv), __fmul_rn(b, inv)), __NV_SATFINITE, __NV_E4M3));
+    return e4m3x2_cvt(__fmul_rn(a, inv), __fmul_rn(b, inv));
+}
+__device__ __forceinline__ uint32_t e4m3x2_div(float a, float b, float s, float inv) {
+    if (isfinite(inv)) {
+        const float qa = __fmul_rn(a, inv), qb = __fmul_rn(b, inv);
+        const uint32_t lo = e4m3x2_cvt(grid_steps(qa, -4), grid_steps(qb, -4));
+        const uint32_t hi = e4m3x2_cvt(grid_steps(qa, 4), grid_steps(qb, 4));
+        if (lo == hi) return lo;
+    }
+    return e4m3x2_cvt(__fdiv_rn(a, s), __fdiv_rn(b, s));
+}
+
+// Eight fp32 values rounded (RN) to bf16 and packed into 16 bytes, f[0] lowest.
+__device__ __forceinline__ uint4 bf16x8(const float *f) {
+    const __nv_bfloat162 p0 = __floats2bfloat162_rn(f[0], f[1]), p1 = __floats2bfloat162_rn(f[2], f[3]);
+    const __nv_bfloat162 p2 = __floats2bfloat162_rn(f[4], f[5]), p3 = __floats2bfloat162_rn(f[6], f[7]);
+    return make_uint4(*reinterpret_cast<const uint32_t *>(&p0), *reinterpret_cast<const uint32_t *>(&p1),
+                      *reinterpret_cast<const uint32_t *>(&p2), *reinterpret_cast<const uint32_t *>(&p3));
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -38,9 +38,10 @@
 // chunks, see remap_tile) is derived on the device from group_offsets, so no
 // host synchronisation is needed.
 //
-// No TMA multicast: every CTA loads its own tiles.  Every wait is bounded (2 s);
-// on expiry the CTA raises MOE_FLAG_TIMEOUT, drains its own outstanding TMA loads
-// and MMAs, frees its TMEM and returns.
+// No TMA multicast: every CTA loads its own tiles.  Every work wait is bounded
+// (by default 2 s, see wait_limit_ns); on expiry the CTA raises MOE_FLAG_TIMEOUT,
+// drains its own outstanding TMA loads and MMAs (waits of up to 2 s each), frees
+// its TMEM and returns.
 #include "tc_util.cuh"
 
 namespace moe {
@@ -160,7 +161,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const __grid_constant__ CUtensorMap tmC,
                     const int32_t *__restrict__ offs, int G, int64_t m_cap, int N, int K,
                     const float *__restrict__ sA, const float *__restrict__ sB, int epi,
-                    void *__restrict__ C, float *__restrict__ sC, int32_t *status) {
+                    void *__restrict__ C, float *__restrict__ sC, int32_t *status, uint64_t wait_ns,
+                    int stall) {
     using Cf = Cfg<PAIR>;
     constexpr int STAGES = Cf::STAGES;
     constexpr uint32_t STAGE_BYTES = Cf::STAGE_BYTES;
@@ -277,8 +279,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const int r1 = swiglu ? I + 128 * tl.nt : BN * tl.nt + 128;  // B rows of columns 128..255
             const int arow = tl.m0 + 128 * static_cast<int>(rank);
             for (int kb = 0; kb < KB; ++kb) {
-                ok = __all_sync(0xffffffffu, mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, status));
+                ok = __all_sync(0xffffffffu, mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, status, false, wait_ns));
                 if (!ok) break;
+                if (!PAIR && stall && blockIdx.x == 0 && t == unit && kb == 0) {
+                    // test hook: CTA 0 never fills its first stage, so the MMA
+                    // warp's wait for it runs out (nothing is in flight for it)
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                    continue;
+                }
                 const uint32_t sa = sbase + stage * STAGE_BYTES;
                 if constexpr (PAIR) {
                     const uint32_t fb = lead_bar0 + 8u * stage;
@@ -297,7 +305,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             }
         }
         // no TMA write may land after the CTAs exit: wait for the last loads
-        // (in a pair the leader's full barriers count both CTAs' bytes)
+        // (in a pair the leader's full barriers count both CTAs' bytes; a stage
+        // skipped by the test hook is the oldest slot and outside this tail,
+        // because `issued` counts real loads only)
         if (leader && lane == 0) {
             const int tail = issued < STAGES ? issued : STAGES;
             for (int i = 0; i < tail; ++i) {
@@ -316,9 +326,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             for (int t = unit; ok && t < num_tiles; t += n_units) {
                 for (int kb = 0; kb < KB; ++kb, ++kc) {
                     const uint32_t buf = kc & 1u, use = kc >> 1;
-                    ok = __all_sync(0xffffffffu, mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, status));
+                    ok = __all_sync(0xffffffffu, mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag, status, false, wait_ns));
                     if (!ok) break;
-                    ok = __all_sync(0xffffffffu, mbar_wait(full_bar(stage), phase, abort_flag, status));
+                    ok = __all_sync(0xffffffffu, mbar_wait(full_bar(stage), phase, abort_flag, status, false, wait_ns));
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t sa = sbase + stage * STAGE_BYTES;
@@ -385,7 +395,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     nb1v = nb1_ok ? __ldg(sb1 + kb + 1) : 0.0f;
                 }
                 const uint32_t buf = kc & 1u, use = kc >> 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(tfull_bar(buf), use & 1u, abort_flag, status))) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, mbar_wait(tfull_bar(buf), use & 1u, abort_flag, status, false, wait_ns))) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -499,12 +509,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 mbar_arrive(xchg_bar(p));
                 uint32_t &xph = p ? xphase1 : xphase0;
                 // warp-uniform outcome: the staged store below is warp-collective
-                if (!__all_sync(0xffffffffu, mbar_wait(xchg_bar(p), xph, abort_flag, status))) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, mbar_wait(xchg_bar(p), xph, abort_flag, status, false, wait_ns))) { ok = false; break; }
                 xph ^= 1u;
                 const float mine = rp[half * 128 + row], other = rp[(half ^ 1) * 128 + row];
                 const bool finite = !isnan(mine) && !isnan(other);
                 const float sc = tile_scale(fmaxf(mine, other), finite);
                 const float inv = __frcp_rn(sc);
+                // codes of fp32(act * (1/scale)): within 1.5 fp32 ulps of the
+                // correctly rounded quotient, so a code can differ from the
+                // division rule's only where act/scale lies that close to an E4M3
+                // rounding boundary (the exact quotient would double the cost of
+                // this tile-end step on the critical path)
                 uint4 v[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -556,32 +571,35 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
 }
 
+// Once per device and tile mode: check the register split and raise the
+// dynamic shared-memory limit.  Returns a moe_status.
 template <bool PAIR>
 static int prepare_kernel() {
-    static int state = 0;   // 0 unknown, 1 ready, 2 unsupported
-    if (state == 0) {
+    static int state[MAX_DEVICES] = {};
+    static std::mutex mu;
+    const int r = once_per_device(state, mu, []() {
         cudaFuncAttributes attr;
-        if (cudaFuncGetAttributes(&attr, grouped_gemm_kernel<PAIR>) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaFuncGetAttributes(&attr, grouped_gemm_kernel<PAIR>) != cudaSuccess) return -MOE_ERR_CUDA;
         // setmaxnreg moves registers inside the launch's allotment: the split
         // 128 x 40 + 256 x 232 must equal 384 x (registers at launch)
-        if (attr.numRegs != LAUNCH_REGS) { state = 2; return MOE_ERR_UNSUPPORTED; }
+        if (attr.numRegs != LAUNCH_REGS) return -MOE_ERR_UNSUPPORTED;
         if (cudaFuncSetAttribute(grouped_gemm_kernel<PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(Cfg<PAIR>::SMEM_BYTES)) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        state = 1;
-    }
-    return state == 1 ? MOE_OK : MOE_ERR_UNSUPPORTED;
+            return -MOE_ERR_CUDA;
+        return 1;
+    });
+    return r > 0 ? MOE_OK : -r;
 }
 
-// Co-resident CTA pairs for one wave of the persistent pair kernel.
-static int pair_clusters(cudaStream_t st) {
-    static int cached = 0;
-    if (cached == 0) {
+// Co-resident CTA pairs for one wave of the persistent pair kernel (per device).
+static int pair_clusters() {
+    static int state[MAX_DEVICES] = {};
+    static std::mutex mu;
+    return once_per_device(state, mu, []() {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(num_sms() / 2 * 2), 1, 1);
         cfg.blockDim = dim3(THREADS, 1, 1);
         cfg.dynamicSmemBytes = Cfg<true>::SMEM_BYTES;
-        cfg.stream = st;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
@@ -590,12 +608,9 @@ static int pair_clusters(cudaStream_t st) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<true>, &cfg) == cudaSuccess && n > 0)
-            cached = n;
-        else
-            cached = num_sms() / 2;
-    }
-    return cached;
+        if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<true>, &cfg) == cudaSuccess && n > 0) return n;
+        return num_sms() / 2;
+    });
 }
 
 }  // namespace gg
@@ -678,13 +693,15 @@ MOE_API int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets
     }
     cudaStream_t st = as_stream(stream);
     const int n = static_cast<int>(N), k = static_cast<int>(K);
+    const uint64_t wait_ns = wait_limit_ns();
+    const int stall = test_stall() ? 1 : 0;
     if (single) {
         grouped_gemm_kernel<false><<<num_sms(), THREADS, Cfg<false>::smem_bytes(G), st>>>(
-            tmA, tmB, tmC, group_offsets, G, m_capacity, n, k, sA, sB, epilogue, C, sC, status);
+            tmA, tmB, tmC, group_offsets, G, m_capacity, n, k, sA, sB, epilogue, C, sC, status, wait_ns, stall);
         return launch_status();
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * pair_clusters(st)), 1, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pair_clusters()), 1, 1);
     cfg.blockDim = dim3(THREADS, 1, 1);
     cfg.dynamicSmemBytes = Cfg<true>::smem_bytes(G);
     cfg.stream = st;
@@ -696,7 +713,7 @@ MOE_API int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<true>, tmA, tmB, tmC, group_offsets, G, m_capacity, n, k, sA, sB,
-                           static_cast<int>(epilogue), C, sC, status) != cudaSuccess)
+                           static_cast<int>(epilogue), C, sC, status, wait_ns, 0) != cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_status();
 }

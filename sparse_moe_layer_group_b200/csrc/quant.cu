@@ -160,7 +160,8 @@ __global__ void __launch_bounds__(256) swiglu_requant_kernel(const float *__rest
         const bool finite = fin_i != 0;
         const float sc = tile_scale(amax, finite);
         const float inv = __frcp_rn(sc);
-        const uint32_t packed = finite ? e4m3x2_rcp(a[0], a[1], inv) | e4m3x2_rcp(a[2], a[3], inv) << 16 : 0x7F7F7F7Fu;
+        const uint32_t packed =
+            finite ? e4m3x2_div(a[0], a[1], sc, inv) | e4m3x2_div(a[2], a[3], sc, inv) << 16 : 0x7F7F7F7Fu;
         q[(row * I + 128 * j) / 4 + lane] = packed;
         if (lane == 0) {
             s[tile] = sc;

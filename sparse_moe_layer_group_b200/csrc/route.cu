@@ -168,7 +168,8 @@ static int launch_select(const moe_dims *d, const float *s_in, const float *part
 
 int router_splits(int T, int E, int H);
 size_t router_tc_ws_bytes(int T, int E, int H);
-int launch_router_tc(const void *x, const float *w, int T, int E, int H, void *ws, float **partial_out,
+int launch_router_split(const float *w, int E, int H, void *pieces_out, cudaStream_t st);
+int launch_router_tc(const void *x, const void *pieces, int T, int E, int H, void *ws, float **partial_out,
                      int *n_split_out, int32_t *status, cudaStream_t st);
 
 size_t route_workspace_bytes(const moe_dims *d) {
@@ -190,9 +191,41 @@ MOE_API int moe_route(const moe_dims *d, const void *x, const float *w_router, c
     if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
     if (!ws || ws_bytes < route_workspace_bytes(d) || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOE_ERR_WORKSPACE;
     cudaStream_t st = as_stream(stream);
+    // the pieces go to the front of the workspace, the partial sums after them
+    rc = launch_router_split(w_router, d->E, d->H, ws, st);
+    if (rc != MOE_OK) return rc;
     float *partial = nullptr;
     int n_split = 0;
-    rc = launch_router_tc(x, w_router, d->T, d->E, d->H, ws, &partial, &n_split, status, st);
+    rc = launch_router_tc(x, ws, d->T, d->E, d->H, ws, &partial, &n_split, status, st);
+    if (rc != MOE_OK) return rc;
+    return launch_select(d, nullptr, partial, n_split, router_offset, scores, e_bias, topk_idx, topk_w, st);
+}
+
+MOE_API size_t moe_router_pieces_bytes(int32_t E, int32_t H) {
+    if (E <= 0 || H <= 0) return 0;
+    return static_cast<size_t>(3) * E * H * 2;
+}
+
+MOE_API int moe_router_split(const float *w_router, int32_t E, int32_t H, void *w_pieces, void *stream) {
+    if (E <= 0 || H <= 0 || H % 128 != 0) return MOE_ERR_INVALID_ARG;
+    if (E > SEL_MAX_E) return MOE_ERR_UNSUPPORTED;
+    if (!w_router || !w_pieces || !aligned16(w_router) || !aligned16(w_pieces)) return MOE_ERR_INVALID_ARG;
+    return launch_router_split(w_router, E, H, w_pieces, as_stream(stream));
+}
+
+MOE_API int moe_route_pieces(const moe_dims *d, const void *x, const void *w_pieces, const float *e_bias,
+                             const float *router_offset, int32_t *topk_idx, float *topk_w, float *scores,
+                             void *ws, size_t ws_bytes, int32_t *status, void *stream) {
+    int rc = check_route_dims(d);
+    if (rc != MOE_OK) return rc;
+    if (d->T == 0) return MOE_OK;
+    if (!x || !w_pieces || !e_bias || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_pieces)) return MOE_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < route_workspace_bytes(d) || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOE_ERR_WORKSPACE;
+    cudaStream_t st = as_stream(stream);
+    float *partial = nullptr;
+    int n_split = 0;
+    rc = launch_router_tc(x, w_pieces, d->T, d->E, d->H, ws, &partial, &n_split, status, st);
     if (rc != MOE_OK) return rc;
     return launch_select(d, nullptr, partial, n_split, router_offset, scores, e_bias, topk_idx, topk_w, st);
 }

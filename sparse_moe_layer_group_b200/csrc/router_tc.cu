@@ -215,27 +215,38 @@ size_t router_tc_ws_bytes(int T, int E, int H) {
     return pieces + part;
 }
 
-// Launch split + tensor-core logits; partial sums land in ws after the pieces.
-int launch_router_tc(const void *x, const float *w, int T, int E, int H, void *ws, float **partial_out,
-                     int *n_split_out, int32_t *status, cudaStream_t st) {
+// W fp32 [E, H] -> three exact bf16 pieces [3, E, H] (the per-weight-set step).
+int launch_router_split(const float *w, int E, int H, void *pieces_out, cudaStream_t st) {
     using namespace rtc;
-    static int prepared = 0;
-    if (!prepared) {
-        if (cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(SMEM_BYTES)) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        prepared = 1;
-    }
-    auto enc = encode_fn();
-    if (!enc) return MOE_ERR_CUDA;
-    uint8_t *base = static_cast<uint8_t *>(ws);
     const size_t piece_elems = static_cast<size_t>(E) * H;
-    __nv_bfloat16 *pieces = reinterpret_cast<__nv_bfloat16 *>(base);
-    float *partial = reinterpret_cast<float *>(base + ((3 * piece_elems * 2 + 255) & ~size_t(255)));
+    __nv_bfloat16 *pieces = reinterpret_cast<__nv_bfloat16 *>(pieces_out);
     const int64_t n4 = static_cast<int64_t>(piece_elems / 4);
     router_split_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(
         reinterpret_cast<const float4 *>(w), reinterpret_cast<uint2 *>(pieces),
         reinterpret_cast<uint2 *>(pieces + piece_elems), reinterpret_cast<uint2 *>(pieces + 2 * piece_elems), n4);
+    return launch_status();
+}
+
+// Tensor-core logits from the pieces; the split-K partial sums land in ws after
+// the space a per-call split would use (so both routes share one workspace size).
+int launch_router_tc(const void *x, const void *pieces_in, int T, int E, int H, void *ws, float **partial_out,
+                     int *n_split_out, int32_t *status, cudaStream_t st) {
+    using namespace rtc;
+    static int state[MAX_DEVICES] = {};
+    static std::mutex mu;
+    const int ready = once_per_device(state, mu, []() {
+        return cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(SMEM_BYTES)) == cudaSuccess
+                   ? 1
+                   : -MOE_ERR_CUDA;
+    });
+    if (ready <= 0) return MOE_ERR_CUDA;
+    auto enc = encode_fn();
+    if (!enc) return MOE_ERR_CUDA;
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    const size_t piece_elems = static_cast<size_t>(E) * H;
+    const void *pieces = pieces_in;
+    float *partial = reinterpret_cast<float *>(base + ((3 * piece_elems * 2 + 255) & ~size_t(255)));
     CUtensorMap tmX, tmW;
     {
         cuuint64_t dims[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
@@ -252,7 +263,7 @@ int launch_router_tc(const void *x, const float *w, int T, int E, int H, void *w
         cuuint64_t strides[2] = {static_cast<cuuint64_t>(H) * 2, static_cast<cuuint64_t>(piece_elems) * 2};
         cuuint32_t box[3] = {BKE, 128, 1};
         cuuint32_t es[3] = {1, 1, 1};
-        if (enc(&tmW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, pieces, dims, strides, box, es,
+        if (enc(&tmW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(pieces), dims, strides, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return MOE_ERR_CUDA;

@@ -1,11 +1,13 @@
 // tcgen05 / TMA / mbarrier helpers shared by the sm_100a tensor-core kernels.
 //
-// All waits are bounded: mbar_wait gives up after WAIT_NS (2 s, %globaltimer),
-// raises MOE_FLAG_TIMEOUT and returns false, so a kernel never spins forever.
+// All waits are bounded: mbar_wait gives up after its limit (by default WAIT_NS
+// = 2 s of %globaltimer), raises MOE_FLAG_TIMEOUT and returns false, so a
+// kernel never spins forever.
 #pragma once
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <stdlib.h>
 
 #include "common.cuh"
 
@@ -32,18 +34,21 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait: false when another role aborted (unless drain is set: the
-// end-of-kernel drains wait out their own 2 s even after an abort) or the 2 s
-// budget ran out.
+// Bounded wait: false when another role aborted (unless drain is set) or the
+// time limit ran out.  A work wait gives up after limit_ns; a drain (drain set:
+// the end-of-kernel waits for the CTA's own TMA loads and MMAs to land) always
+// waits up to WAIT_NS, even after an abort, so that nothing is in flight when
+// the CTA frees its tensor memory and exits.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                       int32_t *status, bool drain = false) {
+                                       int32_t *status, bool drain = false, uint64_t limit_ns = WAIT_NS) {
     if (mbar_try(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
+    const uint64_t limit = drain ? WAIT_NS : limit_ns;
     for (uint32_t n = 1;; ++n) {
         if (mbar_try(bar, parity)) return true;
         if ((n & 63u) == 0) {
             if (!drain && *abort_flag) return false;
-            if (globaltimer() - t0 > WAIT_NS) {
+            if (globaltimer() - t0 > limit) {
                 *abort_flag = 1;
                 set_flag(status, MOE_FLAG_TIMEOUT);
                 return false;
@@ -87,6 +92,18 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *tm,
         "setp.ne.b32 q, %6, 0;\n\t"
         "@q cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n\t}\n"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(bar), "r"(issue)
+        : "memory");
+}
+
+// Plain (untiled) bulk copy global -> this CTA's shared memory, completing on
+// an mbarrier; both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,
+                                          uint32_t issue = 1u) {
+    asm volatile(
+        "{\n\t.reg .pred q;\n\t"
+        "setp.ne.b32 q, %4, 0;\n\t"
+        "@q cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t}\n"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar), "r"(issue)
         : "memory");
 }
 
@@ -257,16 +274,41 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t cta_mask,
         : "memory");
 }
 
+// Limit of the work waits of the grouped GEMM, in nanoseconds: the environment
+// variable MOE_WAIT_LIMIT_NS when set to a number (read at every launch, capped
+// at 60 s), else WAIT_NS.  A short limit makes a wait run out on purpose, which
+// is how the abort path is exercised without any fault.
+inline uint64_t wait_limit_ns() {
+    const char *v = getenv("MOE_WAIT_LIMIT_NS");
+    if (!v || !*v) return WAIT_NS;
+    char *end = nullptr;
+    const unsigned long long n = strtoull(v, &end, 10);
+    if (end == v) return WAIT_NS;
+    return n > 60000000000ull ? 60000000000ull : static_cast<uint64_t>(n);
+}
+
+// The driver's tensor-map encoder, looked up once per process (thread-safe
+// initialisation of a function-local static; the entry point is the same for
+// every device).
+// Testing only: with the environment variable MOE_TEST_STALL=1 (read at every
+// launch) CTA 0 of the one-SM grouped GEMM skips its first operand load, so a
+// work wait runs out at the wait limit and the kernel takes its abort path
+// (MOE_FLAG_TIMEOUT, drain, return) without any fault.
+inline bool test_stall() {
+    const char *v = getenv("MOE_TEST_STALL");
+    return v && v[0] == '1' && v[1] == 0;
+}
+
 inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        return nullptr;
+    }();
     return fn;
 }
 

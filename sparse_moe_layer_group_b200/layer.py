@@ -3,8 +3,9 @@
 PyTorch only allocates device memory and supplies the stream; every step of
 the forward runs in the library's kernels:
 
-  1  moe_route        router GEMM (tensor cores) + sigmoid, group-limited top-K,
-                      gates (3 kernels)
+  1  moe_route_pieces router GEMM (tensor cores, on the bf16 pieces of W_r split
+                      once at construction) + sigmoid, group-limited top-K,
+                      gates (2 kernels)
   2  fp8_quant_1x128  x -> e4m3 codes + 1x128 scales, written straight into the
                       last T rows of the expert-ordered A matrix
   3  moe_permute      stable counting sort by expert + row gather (4 kernels)
@@ -30,7 +31,7 @@ import torch
 
 from . import _abi as abi
 
-LAUNCHES_PER_FORWARD = 11   # 3 route + 1 quant + 4 permute + 2 GEMM + 1 combine
+LAUNCHES_PER_FORWARD = 10   # 2 route + 1 quant + 4 permute + 2 GEMM + 1 combine
 
 
 @dataclass
@@ -87,6 +88,10 @@ class MoELayer:
         self.n_group, self.topk_group, self.rho = n_group, topk_group, rho
         self.d = abi.dims(T, H, E, K, n_group, topk_group, I, rho)
         self.w_router, self.e_bias, self.router_offset = w_router, e_bias, router_offset
+        # the router weights' three exact bf16 pieces, split once (refresh_router
+        # after changing w_router)
+        self.w_pieces = torch.empty(abi.moe_router_pieces_bytes(E, H) // 2, dtype=torch.bfloat16, device=device)
+        self.refresh_router()
         self.qw = weights
         assert weights.E == E, "weights hold E routed experts plus the shared one"
         dev = dict(device=device)
@@ -121,14 +126,15 @@ class MoELayer:
         self.out_f32 = None
         self.status = torch.zeros(1, **i32)
 
-    def forward(self, x: torch.Tensor, out_f32: bool = False, stream=None, gemm1_events=None,
+    def forward(self, x: torch.Tensor, out_f32: bool = False, stream=None, gemm_events=None,
                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
         """x bf16 [T, H] on the device -> out bf16 [T, H] (self.out, or `out` if
         given: a caller-owned contiguous bf16 [T, H] device tensor, e.g. one of
         two buffers while the previous result is still being copied out).
 
-        gemm1_events, if given, is a (start, end) pair of CUDA events recorded
-        around the W13 grouped GEMM on the launching stream."""
+        gemm_events, if given, is a triple of CUDA events recorded on the
+        launching stream before the W13 grouped GEMM, between W13 and W2, and
+        after W2."""
         T, H, E, K, I = self.T, self.H, self.E, self.K, self.I
         if out is None:
             out = self.out
@@ -141,23 +147,30 @@ class MoELayer:
             self.out_f32 = torch.empty(T, H, dtype=torch.float32, device=self.out.device)
         st = self.status
         M = T * K + T
-        abi.moe_route(self.d, x, self.w_router, self.e_bias, self.router_offset, self.topk_idx,
-                      self.topk_w, self.scores, self.ws, st, stream)
+        abi.moe_route_pieces(self.d, x, self.w_pieces, self.e_bias, self.router_offset, self.topk_idx,
+                             self.topk_w, self.scores, self.ws, st, stream)
         abi.fp8_quant_1x128(x, self.xq, self.xs, st, stream)
         abi.moe_permute(self.d, self.topk_idx, self.xq, self.xs, self.load, self.offsets, self.tok_of,
                         self.row_of, self.aq, self.as_, self.ws, st, stream)
         qw = self.qw
-        if gemm1_events is not None:
-            gemm1_events[0].record(torch.cuda.current_stream() if stream is None else stream)
+        ev_stream = torch.cuda.current_stream() if stream is None else stream
+        if gemm_events is not None:
+            gemm_events[0].record(ev_stream)
         abi.fp8_grouped_gemm_blockscaled(E + 1, self.offsets_all, M, 2 * I, H, self.aq, self.as_, qw.w13, qw.s13,
                                          abi.MOE_EPI_SWIGLU_REQUANT, self.actq, self.acts, st, stream)
-        if gemm1_events is not None:
-            gemm1_events[1].record(torch.cuda.current_stream() if stream is None else stream)
+        if gemm_events is not None:
+            gemm_events[1].record(ev_stream)
         abi.fp8_grouped_gemm_blockscaled(E + 1, self.offsets_all, M, H, I, self.actq, self.acts, qw.w2, qw.s2,
                                          abi.MOE_EPI_BF16, self.yperm, None, st, stream)
+        if gemm_events is not None:
+            gemm_events[2].record(ev_stream)
         abi.moe_combine(self.d, self.yperm, self.row_of, self.topk_w, self.ysh, out,
                         self.out_f32 if out_f32 else None, stream)
         return out
+
+    def refresh_router(self, stream=None):
+        """Split the router weights into the pieces the forward routes with."""
+        abi.moe_router_split(self.w_router, self.w_pieces, stream)
 
     def bias_update(self, gamma: float, stream=None, bias: Optional[torch.Tensor] = None):
         """b += gamma * sign(T*K/E - load) from this step's expert loads, into

@@ -8,7 +8,8 @@ import torch
 
 import oracle
 import synth
-from tests._util import TOL_NORMWISE, bf16_ulp, cuda, normwise, np_
+from tests._util import (TOL_NORMWISE, bf16_ulp, cuda, e4m3_boundary_distance, gemm_error_bound, normwise, np_,
+                         swiglu_error_bound)
 
 pytestmark = pytest.mark.gpu
 
@@ -77,8 +78,10 @@ def test_grouped_gemm(lib, sizes, N, K, epi, mode):
     if epi == "bf16":
         r = oracle.round_bf16(r)
     assert normwise(g, r) < TOL_NORMWISE
-    # element-wise: fp32 accumulation error is far below a bf16 ulp
-    tol = 1e-4 * np.abs(r) + 1e-5 * np.abs(r).max() + (bf16_ulp(r) if epi == "bf16" else 0)
+    # element-wise: within the fp32 accumulation bound of the promoted sum (plus
+    # one bf16 rounding for the bf16 epilogue)
+    mag = oracle.grouped_gemm_blockscaled(offs, aq & 0x7F, sa, bq & 0x7F, sb)[:used]
+    tol = gemm_error_bound(mag, K // 128) + (bf16_ulp(r) if epi == "bf16" else 0)
     assert np.all(np.abs(g - r) <= tol)
 
 
@@ -105,33 +108,94 @@ def test_integer_exact_gemm(lib, mode):
     assert np.array_equal(np_(C).astype(np.int64), exact)
 
 
-@pytest.mark.parametrize("sizes,I,K", [([70, 0, 150], 256, 384), ([1], 128, 128), ([300] * 3, 512, 1024),
-                                       ([50, 1100], 256, 256), ([257, 511, 3, 0, 129], 256, 256)])
-@pytest.mark.parametrize("mode", list(TILE_MODES))
-def test_grouped_gemm_swiglu_requant(lib, sizes, I, K, mode):
+SWIGLU_CASES = [([70, 0, 150], 256, 384), ([1], 128, 128), ([300] * 3, 512, 1024), ([50, 1100], 256, 256),
+                ([257, 511, 3, 0, 129], 256, 256)]
+
+
+def _swiglu_gpu(lib, sizes, I, K, mode, seed):
     N = 2 * I
-    a, b, aq, sa, bq, sb, offs, M = _operands(sizes, N, K, seed=91 + I, heavy=False)
+    a, b, aq, sa, bq, sb, offs, M = _operands(sizes, N, K, seed=seed, heavy=False)
     qa, qsa, qb, qsb = _gpu_operands(lib, a, b)
     q = torch.empty(M, I, dtype=torch.uint8, device="cuda")
     s = torch.empty(M, I // 128, dtype=torch.float32, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    lib.fp8_grouped_gemm_blockscaled(len(sizes), cuda(torch.from_numpy(offs)), M, N, K, qa, qsa, qb, qsb,
+    goffs = cuda(torch.from_numpy(offs))
+    lib.fp8_grouped_gemm_blockscaled(len(sizes), goffs, M, N, K, qa, qsa, qb, qsb,
                                      lib.MOE_EPI_SWIGLU_REQUANT | TILE_MODES[mode], q, s, st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
+    return (aq, sa, bq, sb, offs, M), (qa, qsa, qb, qsb, goffs), q, s
+
+
+@pytest.mark.parametrize("sizes,I,K", SWIGLU_CASES)
+@pytest.mark.parametrize("mode", list(TILE_MODES))
+def test_grouped_gemm_swiglu_requant(lib, sizes, I, K, mode):
+    """Fused SwiGLU + 1x128 requant against the oracle, to the bound its error
+    analysis gives: the GPU's gate/up values differ from float64 by at most the
+    fp32 accumulation bound of the promoted GEMM (gemm_error_bound), the act
+    by that propagated through silu(g) u plus the kernel's __expf/__fdividef
+    error (swiglu_error_bound), the tile scale by the act error of the tile's
+    largest element, and the quotient act/scale by both plus 1.5 ulps of the
+    reciprocal.  Every code whose oracle quotient lies farther than that from
+    an E4M3 rounding boundary must be identical; the rest may be a neighbour."""
+    (aq, sa, bq, sb, offs, M), _, q, s = _swiglu_gpu(lib, sizes, I, K, mode, 91 + I)
     gu = oracle.grouped_gemm_blockscaled(offs, aq, sa, bq, sb)
+    mag = oracle.grouped_gemm_blockscaled(offs, aq & 0x7F, sa, bq & 0x7F, sb)
+    eps = gemm_error_bound(mag, K // 128)
     rq, rs, act = oracle.swiglu_requant(gu)
-    gq, gs = np_(q), np_(s)
-    # the scales follow the fp32 amax of act, which differs from float64 by rounding only
-    assert np.max(np.abs(gs - rs) / rs) < 1e-4
-    same = (gq == rq)
-    assert same.mean() > 0.99
+    used = int(offs[-1])
+    gq, gs = np_(q)[:used], np_(s)[:used]
+    rq, rs, act, gu, eps = rq[:used], rs[:used], act[:used], gu[:used], eps[:used]
+    dact = swiglu_error_bound(gu[:, :I], gu[:, I:], eps[:, :I], eps[:, I:])
+    amax = np.abs(act).reshape(used, I // 128, 128).max(-1)
+    damax = dact.reshape(used, I // 128, 128).max(-1)
+    ds = damax / np.maximum(amax, 1e-300) + 2.0 ** -23          # relative scale bound
+    assert np.all(np.abs(gs.astype(np.float64) - rs) <= rs * ds)
+    t = act / np.repeat(rs.astype(np.float64), 128, 1)
+    band = dact / np.repeat(rs.astype(np.float64), 128, 1) + np.abs(t) * (np.repeat(ds, 128, 1) + 2.0 ** -22)
+    outside = e4m3_boundary_distance(t) > band
+    same = gq == rq
+    assert np.all(same[outside]), f"{int((~same & outside).sum())} codes differ away from a rounding boundary"
     deq_g = oracle.dequant_1x128(gq, gs)
     deq_r = oracle.dequant_1x128(rq, rs)
     step = np.abs(deq_r) * 2 ** -3 + np.repeat(rs, 128, 1) * 2 ** -9
-    assert np.all(np.abs(deq_g - deq_r) <= step * 1.01)
-    assert normwise(deq_g, deq_r) < TOL_NORMWISE * 10
-    assert normwise(deq_g, act) < 0.05
+    assert np.all(np.abs(deq_g - deq_r) <= step * (1 + 1e-6))          # the rest: neighbours
+    print(f"identical codes {same.mean():.7f}, band {1 - outside.mean():.2e}")
+    # the band is a worst case; codes actually differ only where the quotient
+    # sits within a few fp32 ulps of a boundary (measured: >= 0.999995 identical)
+    assert same.mean() > 0.9999
+    assert normwise(deq_g, deq_r) < TOL_NORMWISE
+
+
+@pytest.mark.parametrize("sizes,I,K", SWIGLU_CASES[:3])
+def test_fused_requant_matches_division_rule(lib, sizes, I, K):
+    """The fused epilogue requantises with the reciprocal of the tile scale; the
+    stand-alone swiglu_requant divides (the quantisation rule).  Given the same
+    fp32 gate/up values (the F32 epilogue of the same GEMM, whose promotion is
+    the same code), scales agree bit for bit and codes differ only where the
+    quotient lies within 2^-21 of an E4M3 rounding boundary.  Prints the
+    measured mismatch rate."""
+    (aq, sa, bq, sb, offs, M), (qa, qsa, qb, qsb, goffs), q, s = _swiglu_gpu(lib, sizes, I, K, "single", 91 + I)
+    gu = torch.empty(M, 2 * I, dtype=torch.float32, device="cuda")
+    lib.fp8_grouped_gemm_blockscaled(len(sizes), goffs, M, 2 * I, K, qa, qsa, qb, qsb,
+                                     lib.MOE_EPI_F32 | TILE_MODES["single"], gu)
+    qe = torch.empty(M, I, dtype=torch.uint8, device="cuda")
+    se = torch.empty(M, I // 128, dtype=torch.float32, device="cuda")
+    lib.swiglu_requant(gu, qe, se)
+    torch.cuda.synchronize()
+    used = int(offs[-1])
+    assert torch.equal(s[:used], se[:used])
+    diff = (np_(q) != np_(qe))[:used]
+    rate = float(diff.mean())
+    print(f"reciprocal vs division: {int(diff.sum())} of {diff.size} codes differ ({rate:.2e})")
+    if diff.any():
+        g = np_(gu)[:used].astype(np.float64)
+        act32 = oracle.swiglu(g).astype(np.float32).astype(np.float64)   # near-boundary test only
+        t = act32 / np.repeat(np_(se)[:used].astype(np.float64), 128, 1)
+        near = e4m3_boundary_distance(t) <= np.abs(t) * 2.0 ** -21 + swiglu_error_bound(g[:, :I], g[:, I:], 0, 0) / \
+            np.repeat(np_(se)[:used].astype(np.float64), 128, 1)
+        assert np.all(near[diff])
+    assert rate < 1e-4
 
 
 @pytest.mark.parametrize("mode", list(TILE_MODES))

@@ -1,13 +1,15 @@
 """End-to-end layer parity on the GPU (all kernels chained through the C ABI)
-against the float64 oracle: full parity on small shapes, sampled tokens at the
-DeepSeek-V3 shape (T=4096, H=7168, 256+1 experts, top-8, I=2048) and the
-decode shape (T=128) in the launch configuration bench.py times."""
+against the float64 oracle: full parity on small shapes; at the DeepSeek-V3
+shape (T=4096, H=7168, 256+1 experts, top-8, I=2048) and the decode shape
+(T=128), in the launch configuration bench.py times, whole expert segments,
+shared-expert rows and 64 sampled tokens."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import synth
+from tests import _oracle_pool
 from tests._util import TOL_NORMWISE, bf16_ulp, cuda, normwise, np_
 from tests.test_gpu_kernels import check_routing, routing_tol
 
@@ -62,43 +64,104 @@ def test_layer_full_parity(lib, shape):
     assert normwise(np_(layer.ysh), ref["ysh"]) < TOL_NORMWISE
 
 
-def _sampled_parity(lib, shape, T, n_samples, seed):
-    layer, master, wr, b = build_layer(lib, shape, device="cuda", T=T)
-    x = synth.activations(T, shape.H, synth.seed_of(shape, synth.X), shape.x_outlier_frac, device="cuda")
-    out = layer.forward(x)
+def _segment_experts(load, n_top: int = 4) -> list:
+    """Experts whose whole output segments are compared: the n_top most loaded
+    (several M tiles), the most loaded of the rest whose load is not a multiple
+    of 128 (a ragged last M tile) and the least loaded non-empty one."""
+    load = np.asarray(load)
+    order = [int(e) for e in np.argsort(-load, kind="stable") if load[e] > 0]
+    pick = order[:n_top]
+    ragged = [e for e in order if load[e] % 128 != 0 and e not in pick]
+    pick += ragged[:1]
+    rest = [e for e in order[::-1] if e not in pick]
+    pick += rest[:1]
+    return pick
+
+
+def _index_of(sorted_tokens, t) -> int:
+    i = int(np.searchsorted(sorted_tokens, t))
+    assert sorted_tokens[i] == t
+    return i
+
+
+def check_layer_against_oracle(layer, shape, x, wr, b, n_tokens: int, seed: int, offset=None,
+                               segments: bool = True, n_shared_rows: int = 256, out=None):
+    """Full-size parity of one forward already run on `layer` with input x:
+    routing of every token, the expert loads and offsets, the quantised input,
+    whole expert segments of yperm (segments=True), n_shared_rows rows of the
+    shared expert and n_tokens sampled tokens of the output, all against the
+    float64 oracle (expert FFNs evaluated in a process pool)."""
+    T, E, K = x.shape[0], shape.E, shape.K
+    xh = x.float().cpu().numpy()
+    wrh, bh = wr.cpu().numpy(), np.asarray(b.cpu().numpy() if hasattr(b, "cpu") else b)
+    offh = None if offset is None else offset.cpu().numpy()
+    s32 = oracle.router_scores(xh, wrh, offh).astype(np.float32)
+    ridx, rw = oracle.select_experts(s32, bh, shape.n_group, shape.topk_group, K, shape.rho)
+    gidx = np_(layer.topk_idx)
+    same = check_routing(gidx, None, ridx, s32, bh, shape.n_group, shape.topk_group, K,
+                         routing_tol(xh, wrh), min_same=0.97)
+    # gates from the GPU's fp32 affinities (a few ulps from the oracle's)
+    assert np.allclose(np_(layer.topk_w)[same], rw[same], rtol=1e-4, atol=0)
+    load = np_(layer.load)
+    assert load.sum() == T * K
+    assert np.array_equal(np_(layer.offsets), np.concatenate([[0], np.cumsum(load)]))
+    xq, xs = oracle.quant_1x128(xh)
+    assert np.array_equal(np_(layer.xq), xq) and np.array_equal(np_(layer.xs), xs)
+    rload, roffs, rtok, _ = oracle.permute(ridx, E)
+    if same.all():
+        assert np.array_equal(load, rload)
+        assert np.array_equal(np_(layer.tok_of), rtok)
+    rng = np.random.default_rng(seed)
+    seg = _segment_experts(rload) if segments else []
+    pick = np.sort(rng.choice(np.where(same)[0], size=min(n_tokens, int(same.sum())), replace=False))
+    sh_rows = np.sort(rng.choice(T, size=min(n_shared_rows, T), replace=False))
+    toks = {e: set(int(t) for t in rtok[roffs[e]:roffs[e + 1]]) for e in seg}
+    for t in pick:
+        for k in range(K):
+            toks.setdefault(int(ridx[t, k]), set()).add(int(t))
+    toks[-1] = set(int(t) for t in sh_rows) | set(int(t) for t in pick)
+    toks = {e: np.array(sorted(v), dtype=np.int64) for e, v in toks.items()}
+    ys = _oracle_pool.expert_outputs(shape, {e: (xq[v], xs[v]) for e, v in toks.items()},
+                                     device=str(x.device.type))
+    grow = np_(layer.row_of).reshape(T, K)
+    ulp_frac = lambda g, r: float(np.mean(np.abs(g - r) <= bf16_ulp(r)))
+    # whole expert segments (rows of tokens whose routing is identical)
+    for e in seg:
+        st = [int(t) for t in toks[e] if same[t]]
+        rows = [int(grow[t, int(np.where(gidx[t] == e)[0][0])]) for t in st]
+        g = np_(layer.yperm[torch.as_tensor(rows, device=layer.yperm.device)])
+        r = ys[e][[_index_of(toks[e], t) for t in st]]
+        assert normwise(g, r) < TOL_NORMWISE, f"expert {e} (load {rload[e]})"
+        assert ulp_frac(g, r) > 0.99, f"expert {e} (load {rload[e]})"
+    # shared expert rows (both column chunks of its tiles)
+    g = np_(layer.ysh[torch.as_tensor(sh_rows, device=layer.ysh.device)])
+    r = ys[-1][[_index_of(toks[-1], t) for t in sh_rows]]
+    assert normwise(g, r) < TOL_NORMWISE
+    assert ulp_frac(g, r) > 0.99
+    # sampled tokens of the output: the oracle's combine of the oracle's expert rows
+    yk = np.stack([np.stack([ys[int(ridx[t, k])][_index_of(toks[int(ridx[t, k])], t)] for k in range(K)])
+                   for t in pick]).reshape(len(pick) * K, -1)
+    ysh = ys[-1][[_index_of(toks[-1], t) for t in pick]]
+    ref = oracle.round_bf16(oracle.combine(yk, np.arange(len(pick) * K), rw[pick], ysh))
+    got = np_((layer.out if out is None else out)[torch.as_tensor(pick, device=layer.out.device)])
+    assert normwise(got, ref) < TOL_NORMWISE
+    assert ulp_frac(got, ref) > 0.99
+    return same, pick
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("shape", [synth.DSV3, synth.DECODE])
+def test_layer_full_size(lib, shape):
+    """The bench's workloads (DeepSeek-V3 T=4096 and decode T=128) in the launch
+    configuration bench.py times: whole segments of the four most loaded
+    experts, of a ragged one and of the least loaded one, 256 rows of the
+    shared expert and 64 sampled tokens of the output."""
+    layer, master, wr, b = build_layer(lib, shape, device="cuda")
+    x = synth.activations(shape.T, shape.H, synth.seed_of(shape, synth.X), shape.x_outlier_frac, device="cuda")
+    layer.forward(x)
     torch.cuda.synchronize()
     assert int(layer.status.item()) == 0
-    xh = x.float().cpu().numpy()
-    # routing of every token by the oracle (float64 router, fp32 decisions)
-    s32 = oracle.router_scores(xh, wr.cpu().numpy()).astype(np.float32)
-    ridx, rw = oracle.select_experts(s32, b.cpu().numpy(), shape.n_group, shape.topk_group, shape.K, shape.rho)
-    same = check_routing(np_(layer.topk_idx), np_(layer.scores), ridx, s32, b.cpu().numpy(), shape.n_group,
-                         shape.topk_group, shape.K, routing_tol(xh, wr.cpu().numpy()), min_same=0.97)
-    # invariants that hold at any size
-    load = np_(layer.load)
-    assert load.sum() == T * shape.K
-    assert np.array_equal(np_(layer.offsets), np.concatenate([[0], np.cumsum(load)]))
-    # sampled tokens, one by one (rows of every step are independent)
-    rng = np.random.default_rng(seed)
-    cand = np.where(same)[0]
-    pick = np.sort(rng.choice(cand, size=n_samples, replace=False))
-    W = _oracle_weights(master)
-    ref = oracle.moe_forward_tokens(xh[pick], wr.cpu().numpy(), b.cpu().numpy(), W, shape.n_group,
-                                    shape.topk_group, shape.K, shape.rho)
-    assert np.array_equal(ref["idx"], np_(layer.topk_idx)[pick])
-    g = np_(out)[pick]
-    assert normwise(g, ref["out"]) < TOL_NORMWISE
-    assert np.mean(np.abs(g - ref["out"]) <= bf16_ulp(ref["out"])) > 0.99
-
-
-@pytest.mark.slow
-def test_layer_dsv3_sampled_tokens(lib):
-    _sampled_parity(lib, synth.DSV3, synth.DSV3.T, 2, 0)
-
-
-@pytest.mark.slow
-def test_layer_decode_sampled_tokens(lib):
-    _sampled_parity(lib, synth.DECODE, synth.DECODE.T, 2, 1)
+    check_layer_against_oracle(layer, shape, x, wr, b, n_tokens=64, seed=0)
 
 
 def test_layer_single_token(lib):

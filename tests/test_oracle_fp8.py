@@ -154,3 +154,22 @@ def test_quant_128x128_blocks():
             assert int(q[i * 128 + r, j * 128 + c]) & 0x7F == 0x7E
     deq = oracle.dequant_128x128(q, s)
     assert np.abs(deq - w).max() <= np.abs(w).max() * 2 ** -4
+
+
+def test_boundary_helper_matches_the_encoder():
+    """The E4M3 rounding boundaries the GPU parity bands use (tests/_util) are
+    exactly where the oracle's encoder changes code: just below and above every
+    midpoint the codes differ, and the codes of the midpoints' neighbours agree
+    with the nearest representable value."""
+    from tests._util import _MIDPOINTS, e4m3_boundary_distance
+    below = np.nextafter(_MIDPOINTS.astype(np.float32), np.float32(0))
+    above = np.nextafter(_MIDPOINTS.astype(np.float32), np.float32(1e9))
+    assert np.all(oracle.e4m3_encode(below) != oracle.e4m3_encode(above))
+    assert np.all(oracle.e4m3_encode(below) + 1 == oracle.e4m3_encode(above))
+    # no other code change: a fine grid between consecutive midpoints keeps one code
+    rng = np.random.default_rng(0)
+    for lo, hi in zip(_MIDPOINTS[:-1], _MIDPOINTS[1:]):
+        v = rng.uniform(lo, hi, 64).astype(np.float32)
+        v = v[(v > lo) & (v < hi)]
+        assert len(set(oracle.e4m3_encode(v).tolist())) == 1
+    assert e4m3_boundary_distance([1.0625])[0] == 0.0 and e4m3_boundary_distance([1.0])[0] == 0.03125   # 0.96875 and 1.0625
