@@ -216,6 +216,35 @@ int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets, int64_
                                  const uint8_t *B, const float *sB, int32_t epilogue, void *C,
                                  float *sC, int32_t *status, void *stream);
 
+/* Backward pass, weight gradient of the grouped expert GEMMs in FP8 ([repro-guide]
+ * section 3: gemm_wgrad in e4m3 with 1x128 input tiles; [infra-answer]: E4M3
+ * in the forward and the backward pass).  For group g (rows m in
+ * [group_offsets[g], group_offsets[g+1]) of dY [M, N] and X [M, K]):
+ *   dW[g, n, k] = sum_t sdy[t, n] * sx[t, k] * sum_{m in tile t} e4m3(dY[m, n]) e4m3(X[m, k])
+ * The contraction runs over the group's rows, so the 1x128 tiling is taken
+ * along it: tiles of 128 consecutive rows of one column (128x1) that never
+ * cross the group's row range (the last tile of a ragged group is shorter).
+ *
+ * fp8_quant_128x1_grouped quantises x bf16 [M, C] (C % 128 == 0) that way,
+ * with the scale rule of fp8_quant_1x128, and writes the codes TRANSPOSED and
+ * padded: q_t[c, 128 t + r] = code of row r of tile t in column c (tiles
+ * numbered in group order, codes 0 beyond a short tile), uint8 [C, p_capacity];
+ * scales[t, c] fp32 [t_capacity, C].  Capacities: t_capacity >= the number of
+ * tiles (at most ceil(M/128) + G), p_capacity >= 128 * t_capacity and a
+ * multiple of 16.  Offsets that decrease, exceed M or need more tiles than the
+ * capacities raise MOE_FLAG_BAD_OFFSETS and nothing is written.
+ *
+ * fp8_grouped_gemm_wgrad takes two such operands quantised with the same
+ * offsets -- dy_t/sdy from dY (C = N) and x_t/sx from X (C = K) -- and writes
+ * dW fp32 [G, N, K] (an empty group gets zeros); N % 128 == 0, K % 128 == 0,
+ * G <= 2048; fp32 accumulation of each 128-row partial and of the promotion. */
+int fp8_quant_128x1_grouped(const void *x, int64_t M, int64_t C, int32_t G, const int32_t *group_offsets,
+                            uint8_t *q_t, int64_t p_capacity, float *scales, int64_t t_capacity,
+                            int32_t *status, void *stream);
+int fp8_grouped_gemm_wgrad(int32_t G, const int32_t *group_offsets, int64_t M, int64_t N, int64_t K,
+                           const uint8_t *dy_t, const float *sdy, const uint8_t *x_t, const float *sx,
+                           int64_t p_capacity, int64_t t_capacity, float *dW, int32_t *status, void *stream);
+
 /* SwiGLU and 1x128 requantisation of a given fp32 [M, 2I] gate|up matrix
  * (the GEMM epilogue's arithmetic as a stand-alone call; SwiGLU named in
  * [infra-answer], expert intermediate I per [arch-overview]

@@ -63,6 +63,9 @@ _SIGS = {
     "fp8_grouped_gemm_blockscaled": (ctypes.c_int, [_I32, _P, _I64, _I64, _I64, _P, _P, _P, _P, _I32,
                                                     _P, _P, _P, _P]),
     "swiglu_requant": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P]),
+    "fp8_quant_128x1_grouped": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _P, _I64, _P, _I64, _P, _P]),
+    "fp8_grouped_gemm_wgrad": (ctypes.c_int, [_I32, _P, _I64, _I64, _I64, _P, _P, _P, _P, _I64, _I64, _P, _P,
+                                              _P]),
     "moe_combine": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P]),
     "moe_bias_update": (ctypes.c_int, [_I32, _I64, _I32, _F, _P, _P, _P]),
     "moe_balance_stats": (ctypes.c_int, [_DIMS, _P, _P, _P, _I32, ctypes.c_double, _P, _P, _P]),
@@ -184,6 +187,28 @@ def fp8_grouped_gemm_blockscaled(G, group_offsets, m_capacity, N, K, A, sA, B, s
     _check("fp8_grouped_gemm_blockscaled", _lib.fp8_grouped_gemm_blockscaled(
         int(G), _ptr(group_offsets), int(m_capacity), int(N), int(K), _ptr(A), _ptr(sA), _ptr(B), _ptr(sB),
         int(epilogue), _ptr(C), _ptr(sC), _ptr(status), _stream(stream)))
+
+
+def wgrad_capacities(M: int, G: int) -> tuple:
+    """(p_capacity, t_capacity) that fit any grouping of M rows into G groups."""
+    t_cap = (M + 127) // 128 + G
+    return 128 * t_cap, t_cap
+
+
+def fp8_quant_128x1_grouped(x, group_offsets, q_t, scales, status=None, stream=None):
+    M, C = x.shape
+    G = group_offsets.numel() - 1
+    _check("fp8_quant_128x1_grouped", _lib.fp8_quant_128x1_grouped(
+        _ptr(x), M, C, G, _ptr(group_offsets), _ptr(q_t), q_t.shape[1], _ptr(scales), scales.shape[0],
+        _ptr(status), _stream(stream)))
+
+
+def fp8_grouped_gemm_wgrad(group_offsets, M, dy_t, sdy, x_t, sx, dW, status=None, stream=None):
+    G = group_offsets.numel() - 1
+    N, K = dy_t.shape[0], x_t.shape[0]
+    _check("fp8_grouped_gemm_wgrad", _lib.fp8_grouped_gemm_wgrad(
+        G, _ptr(group_offsets), int(M), N, K, _ptr(dy_t), _ptr(sdy), _ptr(x_t), _ptr(sx), dy_t.shape[1],
+        sdy.shape[0], _ptr(dW), _ptr(status), _stream(stream)))
 
 
 def swiglu_requant(gu, q, s, status=None, stream=None):

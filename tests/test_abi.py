@@ -82,3 +82,21 @@ def test_host_validation_rejects_before_launch():
     assert L.swiglu_requant(16, 4, 100, 16, 16, None, None) == a.MOE_ERR_INVALID_ARG
     assert L.moe_bias_update(0, 4, 2, 0.001, 16, 16, None) == a.MOE_ERR_INVALID_ARG
     assert L.moe_combine(None, 16, 16, 16, None, 16, None, None) == a.MOE_ERR_INVALID_ARG
+
+
+def test_wgrad_host_validation():
+    from sparse_moe_layer_group_b200 import _abi as a
+    L = a._lib
+    # columns not a multiple of 128, padded capacity not a multiple of 16
+    assert L.fp8_quant_128x1_grouped(16, 4, 100, 1, 16, 16, 128, 16, 2, None, None) == a.MOE_ERR_INVALID_ARG
+    assert L.fp8_quant_128x1_grouped(16, 4, 128, 1, 16, 16, 130, 16, 2, None, None) == a.MOE_ERR_INVALID_ARG
+    # too many groups; no groups is a no-op
+    assert L.fp8_quant_128x1_grouped(16, 4, 128, 5000, 16, 16, 128, 16, 2, None, None) == a.MOE_ERR_UNSUPPORTED
+    assert L.fp8_grouped_gemm_wgrad(0, None, 0, 128, 128, None, None, None, None, 0, 0, None, None, None) == a.MOE_OK
+    assert L.fp8_grouped_gemm_wgrad(2, 16, 4, 100, 128, 16, 16, 16, 16, 128, 2, 16, None, None) == \
+        a.MOE_ERR_INVALID_ARG
+    assert L.fp8_grouped_gemm_wgrad(5000, 16, 4, 128, 128, 16, 16, 16, 16, 128, 2, 16, None, None) == \
+        a.MOE_ERR_UNSUPPORTED
+    # NULL operands
+    assert L.fp8_grouped_gemm_wgrad(2, 16, 4, 128, 128, None, 16, 16, 16, 128, 2, 16, None, None) == \
+        a.MOE_ERR_INVALID_ARG
