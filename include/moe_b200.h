@@ -263,6 +263,21 @@ int swiglu_requant(const float *gu, int64_t M, int64_t I, uint8_t *q, float *s, 
 int moe_combine(const moe_dims *dims, const void *yperm, const int32_t *row_of,
                 const float *topk_w, const void *yshared, void *out, float *out_f32, void *stream);
 
+/* Expert-parallel placement ([report-walkthrough] section 4.1: experts spread
+ * over devices; tokens dispatched to the devices of their experts and combined
+ * back).  Routed expert e lives on rank e % world as local expert e / world.
+ *   moe_ep_split:   dest_rank[i] = topk_idx[i] % world, local_idx[i] = topk_idx[i] / world
+ *                   for n entries; an index outside [0, E) gets -1 in both and
+ *                   raises MOE_FLAG_BAD_INDEX.
+ *   moe_ep_scatter: out[row_of[i]] = values[i] for the n entries with row_of[i] >= 0
+ *                   (per-pair values into the order of a moe_permute result).
+ * With these, dispatch is moe_permute with the destination ranks as its groups
+ * (rows grouped by rank, (token, slot) order inside each), and the combine of
+ * the returned rows is moe_combine with that permutation's row_of.              */
+int moe_ep_split(const int32_t *topk_idx, int64_t n, int32_t E, int32_t world, int32_t *dest_rank,
+                 int32_t *local_idx, int32_t *status, void *stream);
+int moe_ep_scatter(const int32_t *row_of, const int32_t *values, int64_t n, int32_t *out, void *stream);
+
 /* Sequence-wise balance loss and expert-load entropy ([report-walkthrough]
  * section 3.3: a complementary per-sequence balance loss with a very small
  * coefficient; aux_loss_alpha 0.001 in [repro-guide] section 3).  For each

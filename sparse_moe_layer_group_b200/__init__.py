@@ -10,8 +10,9 @@ from ._abi import (MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_REQUANT, MOE_FLAG_B
                    fp8_grouped_gemm_blockscaled, fp8_quant_128x128, fp8_quant_1x128, moe_bias_update,
                    moe_balance_stats, moe_combine, moe_permute, moe_route, moe_route_pieces, moe_route_select,
                    moe_router_pieces_bytes, moe_router_split, swiglu_requant, fp8_quant_128x1_grouped,
-                   fp8_grouped_gemm_wgrad, wgrad_capacities,
+                   fp8_grouped_gemm_wgrad, wgrad_capacities, moe_ep_split, moe_ep_scatter,
                    workspace_size)
+from .ep import EPMoELayer
 from .layer import LAUNCHES_PER_FORWARD, MoELayer, QuantWeights
 
 __all__ = [

@@ -68,6 +68,8 @@ _SIGS = {
                                               _P]),
     "moe_combine": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P]),
     "moe_bias_update": (ctypes.c_int, [_I32, _I64, _I32, _F, _P, _P, _P]),
+    "moe_ep_split": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P]),
+    "moe_ep_scatter": (ctypes.c_int, [_P, _P, _I64, _P, _P]),
     "moe_balance_stats": (ctypes.c_int, [_DIMS, _P, _P, _P, _I32, ctypes.c_double, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -220,6 +222,16 @@ def swiglu_requant(gu, q, s, status=None, stream=None):
 def moe_combine(d, yperm, row_of, topk_w, yshared, out, out_f32=None, stream=None):
     _check("moe_combine", _lib.moe_combine(ctypes.byref(d), _ptr(yperm), _ptr(row_of), _ptr(topk_w),
                                            _ptr(yshared), _ptr(out), _ptr(out_f32), _stream(stream)))
+
+
+def moe_ep_split(topk_idx, E, world, dest_rank, local_idx, status=None, stream=None):
+    _check("moe_ep_split", _lib.moe_ep_split(_ptr(topk_idx), topk_idx.numel(), int(E), int(world), _ptr(dest_rank),
+                                             _ptr(local_idx), _ptr(status), _stream(stream)))
+
+
+def moe_ep_scatter(row_of, values, out, stream=None):
+    _check("moe_ep_scatter", _lib.moe_ep_scatter(_ptr(row_of), _ptr(values), row_of.numel(), _ptr(out),
+                                                 _stream(stream)))
 
 
 def moe_bias_update(E, T, K, gamma, expert_load, e_bias, stream=None):

@@ -43,11 +43,14 @@ __device__ __forceinline__ void quant_tiles(const uint4 *__restrict__ x, uint2 *
         if (tile >= n_tiles) continue;
         const bool finite = fin_i != 0;
         const float sc = tile_scale(amax, finite);
-        uint32_t lo = 0, hi = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) lo |= static_cast<uint32_t>(quant_code(f[i], sc, finite)) << (8 * i);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) hi |= static_cast<uint32_t>(quant_code(f[4 + i], sc, finite)) << (8 * i);
+        // codes of the correctly rounded quotients v / scale, two at a time
+        // (e4m3x2_div: the product with the reciprocal, confirmed or replaced by
+        // the division wherever it could straddle an E4M3 rounding boundary)
+        const float inv = __frcp_rn(sc);
+        const uint32_t lo = finite ? e4m3x2_div(f[0], f[1], sc, inv) | e4m3x2_div(f[2], f[3], sc, inv) << 16
+                                   : 0x7F7F7F7Fu;
+        const uint32_t hi = finite ? e4m3x2_div(f[4], f[5], sc, inv) | e4m3x2_div(f[6], f[7], sc, inv) << 16
+                                   : 0x7F7F7F7Fu;
         q[tile * 16 + lane16] = make_uint2(lo, hi);
         if (lane16 == 0) {
             scales[tile] = sc;

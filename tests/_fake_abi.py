@@ -1,0 +1,91 @@
+"""A CPU stand-in of the library binding, built from the oracle, for testing host
+logic that chains the calls (the expert-parallel layer's dispatch and combine)
+on CPU ranks without a GPU.  Test infrastructure only.
+
+Every function has the name and arguments of the binding's function and writes
+its outputs in place into CPU tensors; the arithmetic is the oracle's, so a
+chain of these calls reproduces the oracle's layer bit for bit."""
+import numpy as np
+import torch
+
+import oracle
+from sparse_moe_layer_group_b200._abi import MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_REQUANT, dims  # noqa: F401
+
+_WR = {}
+
+
+def workspace_size(d):
+    return 256
+
+
+def moe_router_pieces_bytes(E, H):
+    return 3 * E * H * 2
+
+
+def moe_router_split(w_router, w_pieces, stream=None):
+    _WR[w_pieces.data_ptr()] = w_router.detach().clone()
+
+
+def moe_route_pieces(d, x, w_pieces, e_bias, router_offset, topk_idx, topk_w, scores=None, ws=None,
+                     status=None, stream=None):
+    wr = _WR[w_pieces.data_ptr()].numpy()
+    off = None if router_offset is None else router_offset.numpy()
+    s32 = oracle.router_scores(x.float().numpy(), wr, off).astype(np.float32)
+    idx, w = oracle.select_experts(s32, e_bias.numpy(), d.n_group, d.topk_group, d.K, d.routed_scaling_factor)
+    topk_idx.copy_(torch.from_numpy(idx.astype(np.int32)))
+    topk_w.copy_(torch.from_numpy(w.astype(np.float32)))
+    if scores is not None:
+        scores.copy_(torch.from_numpy(s32))
+
+
+def fp8_quant_1x128(x, q, scales, status=None, stream=None):
+    cq, cs = oracle.quant_1x128(x.float().numpy())
+    q.copy_(torch.from_numpy(cq))
+    scales.copy_(torch.from_numpy(cs))
+
+
+def moe_ep_split(topk_idx, E, world, dest_rank, local_idx, status=None, stream=None):
+    e = topk_idx.reshape(-1).numpy().astype(np.int64)
+    dest_rank.copy_(torch.from_numpy((e % world).astype(np.int32)))
+    local_idx.copy_(torch.from_numpy((e // world).astype(np.int32)))
+
+
+def moe_permute(d, topk_idx, xq, xs, expert_load, expert_offsets, tok_of, row_of, aq, as_, ws, status=None,
+                stream=None):
+    idx = topk_idx.reshape(d.T, d.K).numpy()
+    load, offs, tok, row = oracle.permute(idx, d.E)
+    expert_load.copy_(torch.from_numpy(load))
+    expert_offsets.copy_(torch.from_numpy(offs))
+    tok_of.copy_(torch.from_numpy(tok))
+    row_of.copy_(torch.from_numpy(row))
+    if aq is not None:
+        t = torch.from_numpy(tok.astype(np.int64))
+        aq[:len(tok)].copy_(xq[t])
+        as_[:len(tok)].copy_(xs[t])
+
+
+def moe_ep_scatter(row_of, values, out, stream=None):
+    r = row_of.numpy().astype(np.int64)
+    ok = r >= 0
+    out[torch.from_numpy(r[ok])] = values[torch.from_numpy(ok)]
+
+
+def fp8_grouped_gemm_blockscaled(G, group_offsets, m_capacity, N, K, A, sA, B, sB, epilogue, C, sC=None,
+                                 status=None, stream=None):
+    offs = group_offsets.numpy().astype(np.int64)[:G + 1]
+    used = int(offs[-1])
+    gu = oracle.grouped_gemm_blockscaled(offs, A[:used].numpy(), sA[:used].numpy(), B[:G].numpy(), sB[:G].numpy())
+    lo = int(offs[0])
+    if epilogue == MOE_EPI_SWIGLU_REQUANT:
+        q, s, _ = oracle.swiglu_requant(gu)
+        C[lo:used].copy_(torch.from_numpy(q[lo:used]))
+        sC[lo:used].copy_(torch.from_numpy(s[lo:used]))
+    else:
+        C[lo:used].copy_(torch.from_numpy(oracle.round_bf16(gu[lo:used])).to(C.dtype))
+
+
+def moe_combine(d, yperm, row_of, topk_w, yshared, out, out_f32=None, stream=None):
+    w = topk_w.reshape(d.T, d.K).numpy()
+    ysh = None if yshared is None else yshared.float().numpy()
+    o = oracle.combine(yperm.float().numpy(), row_of.numpy(), w, ysh)
+    out.copy_(torch.from_numpy(oracle.round_bf16(o)).to(out.dtype))

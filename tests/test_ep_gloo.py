@@ -1,0 +1,74 @@
+"""The expert-parallel layer's dispatch, exchange and combine on 2 CPU ranks
+(gloo), with the library calls replaced by their oracle-built CPU stand-ins
+(tests/_fake_abi.py): each rank holds the routed experts e with e % 2 == rank,
+routes its own tokens, and must produce exactly the oracle's single-process
+layer output for those tokens."""
+import os
+import socket
+
+import numpy as np
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    try:
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        import datetime
+        import torch
+        import torch.distributed as dist
+        dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+        import oracle
+        import synth
+        from sparse_moe_layer_group_b200.ep import EPMoELayer
+        from sparse_moe_layer_group_b200.layer import QuantWeights
+        from tests import _fake_abi
+        s = synth.TINY
+        H, E, K, I = s.H, s.E, s.K, s.I
+        T = 24
+
+        def master(kind, e):
+            tid = (synth.SH13 if kind == "w13" else synth.SH2) if e < 0 else (synth.W13 if kind == "w13" else synth.W2)
+            rows, cols = (2 * I, H) if kind == "w13" else (H, I)
+            return synth.expert_weight(rows, cols, s.w_std, synth.seed_of(s, tid, max(e, 0))).float().numpy()
+
+        # this rank's routed experts (global e = l * world + rank) and the shared one, quantised by the oracle
+        mine = [l * world + rank for l in range(E // world)] + [-1]
+        q13 = [oracle.quant_128x128(master("w13", e)) for e in mine]
+        q2 = [oracle.quant_128x128(master("w2", e)) for e in mine]
+        qw = QuantWeights(torch.from_numpy(np.stack([a for a, _ in q13])), torch.from_numpy(np.stack([b for _, b in q13])),
+                          torch.from_numpy(np.stack([a for a, _ in q2])), torch.from_numpy(np.stack([b for _, b in q2])))
+        wr = synth.router_weights(E, H, s.wr_std, synth.seed_of(s, synth.WR))
+        b = synth.expert_bias(E, s.bias_range, synth.seed_of(s, synth.BIAS))
+        x_all = synth.activations(world * T, H, synth.seed_of(s, synth.X))
+        x = x_all[rank * T:(rank + 1) * T].contiguous()
+        layer = EPMoELayer(T, H, E, K, s.n_group, s.topk_group, I, s.rho, wr, b, qw, device="cpu", abi=_fake_abi)
+        out = layer.forward(x).float().numpy()
+        ref = oracle.moe_forward(x.float().numpy(), wr.numpy(), b.numpy(), oracle.LayerWeights(master), s.n_group,
+                                 s.topk_group, K, s.rho)
+        recv = int(layer.recv_counts.sum())
+        dist.destroy_process_group()
+        q.put((rank, bool(np.array_equal(out, ref["out"])), float(np.abs(out - ref["out"]).max()), recv))
+    except Exception as exc:                     # report instead of hanging the parent
+        q.put((rank, False, repr(exc), -1))
+
+
+def test_expert_parallel_layer_matches_the_oracle_on_two_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=300) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+    res.sort()
+    for rank, same, err, recv in res:
+        assert same, f"rank {rank}: {err}"
+        assert recv > 0                      # each rank computed rows for the other rank's tokens too
