@@ -98,6 +98,15 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.path = None
+        self.start = 0          # samples written before the region began
+        self.after = False      # the region held no sample: the next one is used
+
+    def _lines(self) -> int:
+        try:
+            with open(self.path) as f:
+                return f.read().count("\n")
+        except OSError:
+            return 0
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
@@ -108,10 +117,23 @@ class ClockSampler:
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+        # nvidia-smi takes a moment to start: wait (bounded) for its first
+        # sample, so that every sample after `start` falls in the region
+        deadline = time.time() + 10.0
+        while self.proc is not None and self.proc.poll() is None and self._lines() == 0 \
+                and time.time() < deadline:
+            time.sleep(0.02)
+        self.start = self._lines()
         return self
 
     def __exit__(self, *exc):
         if self.proc is not None:
+            # a region shorter than the 200 ms period may hold no sample; then
+            # the first sample after it (at most 200 ms later) stands for it
+            deadline = time.time() + 1.0
+            while self._lines() <= self.start and self.proc.poll() is None and time.time() < deadline:
+                self.after = True
+                time.sleep(0.01)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -121,7 +143,7 @@ class ClockSampler:
     def summary(self) -> dict:
         rows = []
         if self.path and os.path.exists(self.path):
-            for line in open(self.path):
+            for line in open(self.path).readlines()[self.start:]:
                 parts = [p.strip() for p in line.split(",")]
                 if len(parts) >= 9:
                     rows.append(parts)
@@ -133,8 +155,11 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
         loaded = [v for v in sm if mx and v > 0.5 * max(mx)] or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+        out = {"sm_mhz": statistics.median(loaded) if loaded else None,
+               "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+        if self.after:
+            out["window"] = "region shorter than the 200 ms sampling period: the first sample after it"
+        return out
 
 
 # ----------------------------------------------------------------- GPU arm
@@ -243,7 +268,6 @@ def run_gpu(args, rank, world, local):
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
-        time.sleep(0.3)            # let the sampler start before the timed region
         t0.record(stream)
         for _ in range(args.steps):
             step(record=True)
@@ -360,7 +384,7 @@ def run_gpu(args, rank, world, local):
         "balance": balance,
     }
     if world == 1 and not args.no_workloads:
-        rec["workloads"] = run_workloads(layer.qw, pk, pk_kind)
+        rec["workloads"] = run_workloads(layer.qw, pk, pk_kind, layer.offsets_all)
     return rec
 
 
@@ -489,10 +513,70 @@ def leg_gemm_dense(pk, M: int = 4096, N: int = 18432, K: int = 7168, iters: int 
             "l2": "flushed before every launch (256 MB write)"}
 
 
-def run_workloads(qw, pk, pk_kind) -> dict:
+def leg_wgrad(offsets_all, pk, iters: int = 5) -> dict:
+    """Backward weight gradient of W13 at the DeepSeek-V3 layer shape: dW13 [257,
+    2I, H] = dY^T X per expert over the layer's own expert segments (the T*K
+    routed rows in expert order, then the T shared rows), dY bf16 [T*K + T, 2I]
+    and X bf16 [T*K + T, H] seeded N(0,1); one step = the two 128x1 quantisations
+    and the wgrad GEMM.  Bound by HBM: the fp32 gradient alone is 30 GB."""
+    import sparse_moe_layer_group_b200 as moe
+    abi = moe.abi
+    s = synth.DSV3
+    H, I = s.H, s.I
+    offs = offsets_all
+    G = offs.numel() - 1
+    M = int(offs[-1].item())
+    dy = synth.normal((M, 2 * I), 1.0, 81, device="cuda", dtype=torch.bfloat16)
+    x = synth.activations(M, H, 82, device="cuda")
+    p_cap, t_cap = abi.wgrad_capacities(M, G)
+    dq = torch.empty(2 * I, p_cap, dtype=torch.uint8, device="cuda")
+    ds = torch.empty(t_cap, 2 * I, dtype=torch.float32, device="cuda")
+    xq = torch.empty(H, p_cap, dtype=torch.uint8, device="cuda")
+    xs = torch.empty(t_cap, H, dtype=torch.float32, device="cuda")
+    dW = torch.empty(G, 2 * I, H, dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def step(ev=None):
+        abi.fp8_quant_128x1_grouped(dy, offs, dq, ds, st)
+        abi.fp8_quant_128x1_grouped(x, offs, xq, xs, st)
+        if ev is not None:
+            ev[0].record()
+        abi.fp8_grouped_gemm_wgrad(offs, M, dq, ds, xq, xs, dW, st)
+        if ev is not None:
+            ev[1].record()
+
+    step()
+    torch.cuda.synchronize()
+    evs = []
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(iters):
+        ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        evs.append(ev)
+        step(ev)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / iters
+    g_ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+    flops = 2.0 * M * 2 * I * H
+    out_bytes = G * 2 * I * H * 4
+    in_bytes = (2 * I + H) * (p_cap + 4 * t_cap)
+    status = int(st.item())
+    del dy, x, dq, ds, xq, xs, dW
+    torch.cuda.empty_cache()
+    return {"workload": f"wgrad of W13 at the DSV3 layer shape: {G} groups (256 routed + shared), {M} rows, "
+                        f"dW fp32 [{G}, {2 * I}, {H}]", "iters": iters, "ms_per_step": round(ms, 4),
+            "gemm_ms": round(g_ms, 4), "gemm_tflops": round(flops / g_ms / 1e9, 1),
+            "gemm_gbs": round((out_bytes + in_bytes) / g_ms / 1e6, 1),
+            "gemm_frac_of_hbm": round((out_bytes + in_bytes) / g_ms / 1e6 / pk["hbm_gbs"], 3),
+            "algorithmic_bytes": out_bytes + in_bytes, "device_status": status}
+
+
+def run_workloads(qw, pk, pk_kind, offsets_all=None) -> dict:
     """The other configurations of the layer, each timed with CUDA events only:
     prefill with skewed routing, decode, and the dense GEMM sweep's largest
-    compute-bound shape.  The layer legs reuse the resident DeepSeek-V3 expert
+    compute-bound shape, and the backward wgrad of W13 over the DSV3 step's own
+    expert segments.  The layer legs reuse the resident DeepSeek-V3 expert
     weights (same sizes); their routers and inputs come from their own seeds."""
     # the dense GEMM first, after a short idle: run after the long prefill leg it
     # would be timed at power-capped clocks against the burst peak
@@ -501,6 +585,8 @@ def run_workloads(qw, pk, pk_kind) -> dict:
         dense = leg_gemm_dense(pk)
     dense["clocks"] = clk.summary()
     out = {"gemm_dense": dense, "prefill_skew": leg_prefill(qw, pk), "decode": leg_decode(qw, pk)}
+    if offsets_all is not None:
+        out["wgrad"] = leg_wgrad(offsets_all, pk)
     torch.cuda.empty_cache()
     return out
 

@@ -40,12 +40,15 @@ constexpr uint32_t A_BYTES = 128 * 128;      // 128 rows of dY^T x one tile of 1
 constexpr uint32_t B_BYTES = 256 * 128;      // 256 rows of X^T
 constexpr uint32_t SX_BYTES = 256 * 4;       // the tile's column scales of X
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SX_BYTES;   // 49 KB, 1 KB aligned
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;
 constexpr int THREADS = 384;
 constexpr int EPI_THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int LAUNCH_REGS = 168;
-constexpr uint32_t OFF_BARS = STAGES * STAGE_BYTES;
+constexpr uint32_t EPI_BOX = 32 * 128;          // one TMA-store box: 32 rows x 32 fp32, 128-byte swizzle
+constexpr uint32_t EPI_STG = 2 * EPI_BOX;       // per epilogue warp: two boxes in flight
+constexpr uint32_t OFF_EPI = STAGES * STAGE_BYTES;
+constexpr uint32_t OFF_BARS = OFF_EPI + 8 * EPI_STG;
 constexpr uint32_t OFF_MISC = OFF_BARS + 128;
 constexpr uint32_t OFF_TSTART = OFF_MISC + 32;   // int32 [G + 1]
 constexpr uint32_t SMEM_BYTES = OFF_TSTART + (MAX_G + 1) * 4 + 1024;
@@ -79,14 +82,18 @@ __device__ __forceinline__ void group_tiles(const int32_t *__restrict__ offs, in
 }
 
 // ---------------------------------------------------------------- quantiser
-// CTA = (tile t, 128 columns); thread (column c, half h) owns rows 64h..64h+63
-// of the tile in column c.
+// CTA = (tile t, a strided set of 128-column blocks: gridDim.y of them apart),
+// so the group-table scan is paid once per several blocks.  Each 128 x 128 bf16
+// block is staged in shared memory with 16-byte loads (eight per thread, all
+// issued before use); then thread (column c, half h) owns rows 64h..64h+63 of
+// column c.
 __global__ void __launch_bounds__(256) quant_128x1_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t C,
                                                           const int32_t *__restrict__ offs, int G,
                                                           uint8_t *__restrict__ q_t, int64_t p_cap,
                                                           float *__restrict__ scales, int64_t t_cap,
                                                           int32_t *status) {
     __shared__ int32_t tstart[MAX_G + 1];
+    __shared__ __align__(16) uint16_t blk[128 * 128];   // the tile's rows x 128 columns
     __shared__ float s_amax[2][128];
     __shared__ int s_fin[2][128];
     __shared__ int bad;
@@ -112,14 +119,32 @@ __global__ void __launch_bounds__(256) quant_128x1_kernel(const uint16_t *__rest
     const int64_t r1 = min(r0 + 128, static_cast<int64_t>(__ldg(offs + g + 1)));
     const int nrows = static_cast<int>(r1 - r0);
     const int cl = tid & 127, h = tid >> 7;
-    const int64_t c = static_cast<int64_t>(blockIdx.y) * 128 + cl;
+    for (int64_t cb = blockIdx.y; cb < C / 128; cb += gridDim.y) {
+    const int64_t c0 = cb * 128;
+    const int64_t c = c0 + cl;
+    __syncthreads();   // the previous block's reads of blk and s_amax are done
+    {
+        // 128 rows x 256 bytes: 16 lanes per row, 16 rows per pass, 8 passes
+        uint4 ld[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const int r = 16 * p + (tid >> 4), seg = tid & 15;
+            ld[p] = r < nrows ? __ldg(reinterpret_cast<const uint4 *>(x + (r0 + r) * C + c0) + seg)
+                              : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const int r = 16 * p + (tid >> 4), seg = tid & 15;
+            reinterpret_cast<uint4 *>(blk + r * 128)[seg] = ld[p];
+        }
+    }
+    __syncthreads();
     float v[64];
     float amax = 0.0f;
     bool fin = true;
 #pragma unroll
     for (int i = 0; i < 64; ++i) {
-        const int r = 64 * h + i;
-        v[i] = r < nrows ? __uint_as_float(static_cast<uint32_t>(__ldg(x + (r0 + r) * C + c)) << 16) : 0.0f;
+        v[i] = __uint_as_float(static_cast<uint32_t>(blk[(64 * h + i) * 128 + cl]) << 16);
         amax_step(v[i], amax, fin);
     }
     s_amax[h][cl] = amax;
@@ -146,6 +171,7 @@ __global__ void __launch_bounds__(256) quant_128x1_kernel(const uint16_t *__rest
         scales[static_cast<int64_t>(t) * C + c] = sc;
         if (!finite) set_flag(status, MOE_FLAG_NONFINITE);
     }
+    }
 }
 
 // ---------------------------------------------------------------- GEMM
@@ -167,7 +193,7 @@ __device__ __forceinline__ Tile decode(int t, int NTn, int NTk, const int32_t *t
 
 __global__ void __launch_bounds__(THREADS, 1)
 wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-             const int32_t *__restrict__ offs, int G, int64_t M, int N, int K, const float *__restrict__ sdy,
+             const __grid_constant__ CUtensorMap tmD, const int32_t *__restrict__ offs, int G, int64_t M, int N, int K, const float *__restrict__ sdy,
              const float *__restrict__ sx, int64_t t_cap, int64_t p_cap, float *__restrict__ dW, int32_t *status,
              uint64_t wait_ns) {
     extern __shared__ uint8_t smem_raw[];
@@ -203,6 +229,7 @@ wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     } else if (warp == 3 && lane == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmD)) : "memory");
     }
     if (warp == 1) {
         __syncwarp();
@@ -352,11 +379,34 @@ wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             if (!ok) break;
             const int k = tl.k0 + 128 * half;
             if (k < K) {
-                float4 *d = reinterpret_cast<float4 *>(dW + (static_cast<int64_t>(tl.g) * N + n) * K + k);
+                // the warp's 32 rows (n0 + 32 q ..) x this half's 128 columns as four
+                // 32 x 32 fp32 TMA-store boxes from two alternating staging boxes (row r's
+                // 16-byte chunk i at i ^ (r % 8): the 128-byte swizzle)
+                uint8_t *stg = smem + OFF_EPI + (warp - 4) * EPI_STG;
+                const uint32_t stg_s = sbase + OFF_EPI + (warp - 4) * EPI_STG;
+                const int32_t drow = tl.g * N + tl.n0 + 32 * q;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) d[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t bsel = (c & 1) * EPI_BOX;
+                    if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float *f = acc + 32 * c + 4 * i;
+                        *reinterpret_cast<uint4 *>(stg + bsel + lane * 128 + ((i ^ (lane & 7)) << 4)) =
+                            make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                                       __float_as_uint(f[3]));
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    tma_store_2d(&tmD, stg_s + bsel, k + 32 * c, drow, lane == 0 ? 1u : 0u);
+                    if (lane == 0) bulk_commit();
+                }
             }
         }
+        // this warp's TMA stores are complete before the CTA exits
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -397,7 +447,8 @@ MOE_API int fp8_quant_128x1_grouped(const void *x, int64_t M, int64_t C, int32_t
     if (G == 0 || C == 0 || t_capacity == 0) return MOE_OK;
     if (G > wg::MAX_G || t_capacity > 0x7fffffffLL || C / 128 > 65535) return MOE_ERR_UNSUPPORTED;
     if (!x || !group_offsets || !q_t || !scales || !aligned16(x) || !aligned16(q_t)) return MOE_ERR_INVALID_ARG;
-    dim3 grid(static_cast<unsigned>(t_capacity), static_cast<unsigned>(C / 128), 1);
+    const int64_t cblocks = C / 128;
+    dim3 grid(static_cast<unsigned>(t_capacity), static_cast<unsigned>(cblocks < 8 ? cblocks : 8), 1);
     wg::quant_128x1_kernel<<<grid, 256, 0, as_stream(stream)>>>(
         static_cast<const uint16_t *>(x), M, C, group_offsets, G, q_t, p_capacity, scales, t_capacity, status);
     return launch_status();
@@ -412,7 +463,8 @@ MOE_API int fp8_grouped_gemm_wgrad(int32_t G, const int32_t *group_offsets, int6
     if (N % 128 != 0 || K % 128 != 0 || p_capacity % 16 != 0) return MOE_ERR_INVALID_ARG;
     if (G == 0 || N == 0 || K == 0) return MOE_OK;
     if (G > MAX_G || N > 0x7fffffffLL || K > 0x7fffffffLL || p_capacity > 0x7fffffffLL ||
-        static_cast<int64_t>(G) * (N / 128) * ((K + BN - 1) / BN) > 0x7fffffffLL)
+        static_cast<int64_t>(G) * (N / 128) * ((K + BN - 1) / BN) > 0x7fffffffLL ||
+        static_cast<int64_t>(G) * N > 0x7fffffffLL)
         return MOE_ERR_UNSUPPORTED;
     if (!group_offsets || !dy_t || !sdy || !x_t || !sx || !dW) return MOE_ERR_INVALID_ARG;
     if (p_capacity == 0) return MOE_ERR_INVALID_ARG;
@@ -444,8 +496,19 @@ MOE_API int fp8_grouped_gemm_wgrad(int32_t G, const int32_t *group_offsets, int6
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return MOE_ERR_CUDA;
     }
+    CUtensorMap tmD;   // dW viewed as [G * N rows, K] fp32, stored in 32 x 32 boxes
+    {
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(G) * static_cast<cuuint64_t>(N)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 4};
+        cuuint32_t box[2] = {32, 32};
+        cuuint32_t es[2] = {1, 1};
+        if (enc(&tmD, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dW, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MOE_ERR_CUDA;
+    }
     wgrad_kernel<<<num_sms(), THREADS, SMEM_BYTES, as_stream(stream)>>>(
-        tmA, tmB, group_offsets, G, M, static_cast<int>(N), static_cast<int>(K), sdy, sx, t_capacity, p_capacity, dW,
+        tmA, tmB, tmD, group_offsets, G, M, static_cast<int>(N), static_cast<int>(K), sdy, sx, t_capacity, p_capacity, dW,
         status, wait_limit_ns());
     return launch_status();
 }
