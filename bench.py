@@ -226,11 +226,12 @@ def recorded_w13_traffic(algorithmic_bytes: int):
 
 def gemm1_bytes(layer, touched: int) -> int:
     """Algorithmic HBM bytes of the W13 grouped GEMM launch: W13 of the touched
-    routed experts and of the shared expert, the T*K + T A rows (codes +
-    scales) and the requantised output rows (codes + scales)."""
+    routed experts and of the shared expert, the A rows it reads (codes +
+    scales: the T token rows when it gathers them, else the T*K + T rows of the
+    permuted copy) and the requantised output rows (codes + scales)."""
     T, H, K, I = layer.T, layer.H, layer.K, layer.I
     w = (touched + 1) * (2 * I * H + (2 * I // 128) * (H // 128) * 4)
-    a = (T * K + T) * (H + (H // 128) * 4)
+    a = (T if layer.gather else T * K + T) * (H + (H // 128) * 4)
     o = (T * K + T) * (I + (I // 128) * 4)
     return w + a + o
 
@@ -260,7 +261,7 @@ def run_gpu(args, rank, world, local):
         # workload keeps the configured routing bias b = 0
         layer.bias_update(gamma, bias=b_next)
 
-    launches_per_step = moe.LAUNCHES_PER_FORWARD + 1
+    launches_per_step = layer.launches_per_forward + 1
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -384,7 +385,7 @@ def run_gpu(args, rank, world, local):
         "balance": balance,
     }
     if world == 1 and not args.no_workloads:
-        rec["workloads"] = run_workloads(layer.qw, pk, pk_kind, layer.offsets_all)
+        rec["workloads"] = run_workloads(layer.qw, pk, pk_kind, layer.offsets_all, layer)
     return rec
 
 
@@ -572,7 +573,46 @@ def leg_wgrad(offsets_all, pk, iters: int = 5) -> dict:
             "algorithmic_bytes": out_bytes + in_bytes, "device_status": status}
 
 
-def run_workloads(qw, pk, pk_kind, offsets_all=None) -> dict:
+def leg_gather(layer, pk, iters: int = 10) -> dict:
+    """W13 of the DeepSeek-V3 step two ways on the step's own routing: over the
+    materialised permuted rows (the layer's default, as timed in the step) and
+    with the routed rows fetched through tok_of by TMA row gathers (the fused
+    dispatch variant, which drops the permute's row-copy kernel and its
+    T*K x H copy)."""
+    import sparse_moe_layer_group_b200 as moe
+    abi = moe.abi
+    T, H, K, I, E = layer.T, layer.H, layer.K, layer.I, layer.E
+    M = T * K + T
+    qw = layer.qw
+    a_map = torch.cat([layer.tok_of, torch.arange(T, dtype=torch.int32, device="cuda")])
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def plain():
+        abi.fp8_grouped_gemm_blockscaled(E + 1, layer.offsets_all, M, 2 * I, H, layer.aq, layer.as_, qw.w13, qw.s13,
+                                         abi.MOE_EPI_SWIGLU_REQUANT, layer.actq, layer.acts, st)
+
+    def gather():
+        abi.fp8_grouped_gemm_blockscaled_gather(E + 1, layer.offsets_all, M, 2 * I, H, layer.xq, layer.xs, a_map,
+                                                qw.w13, qw.s13, abi.MOE_EPI_SWIGLU_REQUANT, layer.actq, layer.acts,
+                                                st)
+
+    out = {"workload": "W13 grouped GEMM of the DSV3 step (T=4096, 257 groups, 36864 rows): materialised "
+                       "permuted A vs A rows gathered through tok_of (tile::gather4)", "iters": iters}
+    for name, fn in (("materialised_ms", plain), ("gather_ms", gather)):
+        fn()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record()
+        for _ in range(iters):
+            fn()
+        ev[1].record()
+        torch.cuda.synchronize()
+        out[name] = round(ev[0].elapsed_time(ev[1]) / iters, 4)
+    out["device_status"] = int(st.item())
+    return out
+
+
+def run_workloads(qw, pk, pk_kind, offsets_all=None, layer=None) -> dict:
     """The other configurations of the layer, each timed with CUDA events only:
     prefill with skewed routing, decode, and the dense GEMM sweep's largest
     compute-bound shape, and the backward wgrad of W13 over the DSV3 step's own
@@ -587,6 +627,8 @@ def run_workloads(qw, pk, pk_kind, offsets_all=None) -> dict:
     out = {"gemm_dense": dense, "prefill_skew": leg_prefill(qw, pk), "decode": leg_decode(qw, pk)}
     if offsets_all is not None:
         out["wgrad"] = leg_wgrad(offsets_all, pk)
+    if layer is not None and not layer.gather:
+        out["gather"] = leg_gather(layer, pk)
     torch.cuda.empty_cache()
     return out
 

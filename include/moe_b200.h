@@ -216,6 +216,27 @@ int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets, int64_
                                  const uint8_t *B, const float *sB, int32_t epilogue, void *C,
                                  float *sC, int32_t *status, void *stream);
 
+/* fp8_grouped_gemm_blockscaled with the A rows gathered through a row map
+ * instead of stored in group order ([report-walkthrough] sections 3.2 and 4.1:
+ * the routed rows are dispatched to their experts; gathering them inside the
+ * GEMM leaves the result unchanged and never writes the permuted copy):
+ *   row m of group g reads A row a_map[m] and its scales sA[a_map[m], :],
+ *   i.e. C[m, n] = sum_kb sA[a_map[m], kb] * sB[g, n/128, kb] *
+ *                  sum_{k in kb} e4m3(A[a_map[m], k]) * e4m3(B[g, n, k])
+ *   A  e4m3 [a_rows, K] (16-byte aligned);  sA fp32 [a_rows, K/128]
+ *   a_map device int32 [m_capacity]; entries of rows outside every group are
+ *   not read.  An entry outside [0, a_rows) raises MOE_FLAG_BAD_INDEX and that
+ *   output row is unspecified (nothing is read outside A).  a_rows >= 1.
+ * Everything else (groups, B, epilogues, C, limits) as fp8_grouped_gemm_blockscaled;
+ * the call always runs one-SM tiles (MOE_GEMM_PAIR_CTA is ignored).  In the
+ * layer, A is the T quantised token rows and a_map the permutation's tok_of
+ * followed by 0..T-1 for the shared expert's group.                         */
+int fp8_grouped_gemm_blockscaled_gather(int32_t G, const int32_t *group_offsets, int64_t m_capacity,
+                                        int64_t N, int64_t K, const uint8_t *A, const float *sA,
+                                        int64_t a_rows, const int32_t *a_map, const uint8_t *B,
+                                        const float *sB, int32_t epilogue, void *C, float *sC,
+                                        int32_t *status, void *stream);
+
 /* Backward pass, weight gradient of the grouped expert GEMMs in FP8 ([repro-guide]
  * section 3: gemm_wgrad in e4m3 with 1x128 input tiles; [infra-answer]: E4M3
  * in the forward and the backward pass).  For group g (rows m in

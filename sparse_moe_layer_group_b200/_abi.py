@@ -62,6 +62,8 @@ _SIGS = {
     "moe_permute_noalloc_max_scratch": (_SZ, []),
     "fp8_grouped_gemm_blockscaled": (ctypes.c_int, [_I32, _P, _I64, _I64, _I64, _P, _P, _P, _P, _I32,
                                                     _P, _P, _P, _P]),
+    "fp8_grouped_gemm_blockscaled_gather": (ctypes.c_int, [_I32, _P, _I64, _I64, _I64, _P, _P, _I64, _P, _P, _P,
+                                                           _I32, _P, _P, _P, _P]),
     "swiglu_requant": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P]),
     "fp8_quant_128x1_grouped": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _P, _I64, _P, _I64, _P, _P]),
     "fp8_grouped_gemm_wgrad": (ctypes.c_int, [_I32, _P, _I64, _I64, _I64, _P, _P, _P, _P, _I64, _I64, _P, _P,
@@ -189,6 +191,14 @@ def fp8_grouped_gemm_blockscaled(G, group_offsets, m_capacity, N, K, A, sA, B, s
     _check("fp8_grouped_gemm_blockscaled", _lib.fp8_grouped_gemm_blockscaled(
         int(G), _ptr(group_offsets), int(m_capacity), int(N), int(K), _ptr(A), _ptr(sA), _ptr(B), _ptr(sB),
         int(epilogue), _ptr(C), _ptr(sC), _ptr(status), _stream(stream)))
+
+
+def fp8_grouped_gemm_blockscaled_gather(G, group_offsets, m_capacity, N, K, A, sA, a_map, B, sB, epilogue, C,
+                                        sC=None, status=None, stream=None):
+    """A: e4m3 [a_rows, K] source rows, a_map int32 [m_capacity] (GEMM row -> A row)."""
+    _check("fp8_grouped_gemm_blockscaled_gather", _lib.fp8_grouped_gemm_blockscaled_gather(
+        int(G), _ptr(group_offsets), int(m_capacity), int(N), int(K), _ptr(A), _ptr(sA), int(A.shape[0]),
+        _ptr(a_map), _ptr(B), _ptr(sB), int(epilogue), _ptr(C), _ptr(sC), _ptr(status), _stream(stream)))
 
 
 def wgrad_capacities(M: int, G: int) -> tuple:

@@ -38,6 +38,17 @@
 // chunks, see remap_tile) is derived on the device from group_offsets, so no
 // host synchronisation is needed.
 //
+// Gather variant (template parameter GATHER, single tiles only): A is not given
+// in group order but as the source rows it is made of, with a map from GEMM row
+// m to source row a_map[m] (the layer's permutation: A row m of expert g is
+// token tok_of[m]'s quantised activation row), so the permuted copy of the
+// activations is never written.  The producer warp loads each stage's A tile
+// with 32 TMA row gathers (tile::gather4), one per lane: lane l fetches tile rows
+// 4l..4l+3 (their source rows read from a_map once per tile) into bytes
+// 512l..512l+511 of the tile, in the same 128-byte swizzle as a tiled load.  Rows
+// outside the group read source row 0 (computed, never stored).  The epilogue
+// reads the A row scales through the same map.
+//
 // No TMA multicast: every CTA loads its own tiles.  Every work wait is bounded
 // (by default 2 s, see wait_limit_ns); on expiry the CTA raises MOE_FLAG_TIMEOUT,
 // drains its own outstanding TMA loads and MMAs (waits of up to 2 s each), frees
@@ -155,14 +166,15 @@ __device__ __forceinline__ int remap_tile(int v, int R, int S, int C) {
     return v;
 }
 
-template <bool PAIR>
+template <bool PAIR, bool GATHER>
 __global__ void __launch_bounds__(THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC,
                     const int32_t *__restrict__ offs, int G, int64_t m_cap, int N, int K,
                     const float *__restrict__ sA, const float *__restrict__ sB, int epi,
                     void *__restrict__ C, float *__restrict__ sC, int32_t *status, uint64_t wait_ns,
-                    int stall) {
+                    int stall, const int32_t *__restrict__ a_map, int64_t a_rows) {
+    static_assert(!(PAIR && GATHER), "the gather variant runs single tiles");
     using Cf = Cfg<PAIR>;
     constexpr int STAGES = Cf::STAGES;
     constexpr uint32_t STAGE_BYTES = Cf::STAGE_BYTES;
@@ -278,6 +290,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const int r0 = swiglu ? 128 * tl.nt : BN * tl.nt;            // B rows of columns 0..127
             const int r1 = swiglu ? I + 128 * tl.nt : BN * tl.nt + 128;  // B rows of columns 128..255
             const int arow = tl.m0 + 128 * static_cast<int>(rank);
+            int src[4] = {0, 0, 0, 0};   // gather: source rows of tile rows 4 lane .. 4 lane + 3
+            if (GATHER) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int m = tl.m0 + 4 * lane + i;
+                    if (m < tl.m_end) {
+                        const int v = __ldg(a_map + m);
+                        if (v >= 0 && v < a_rows) src[i] = v;
+                        else set_flag(status, MOE_FLAG_BAD_INDEX);
+                    }
+                }
+            }
             for (int kb = 0; kb < KB; ++kb) {
                 ok = __all_sync(0xffffffffu, mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, status, false, wait_ns));
                 if (!ok) break;
@@ -295,7 +319,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     tma_load_3d_pair(sa + A_BYTES, &tmB, kb * BK, leader ? r0 : r1, tl.g, fb, one);
                 } else {
                     mbar_expect_tx_if(full_bar(stage), STAGE_BYTES, one);
-                    tma_load_2d(sa, &tmA, kb * BK, arow, full_bar(stage), one);
+                    if (GATHER)
+                        tma_gather4(sa + 512u * lane, &tmA, kb * BK, src[0], src[1], src[2], src[3], full_bar(stage));
+                    else
+                        tma_load_2d(sa, &tmA, kb * BK, arow, full_bar(stage), one);
                     tma_load_3d(sa + A_BYTES, &tmB, kb * BK, r0, tl.g, full_bar(stage), one);
                     tma_load_3d(sa + A_BYTES + B_HALF, &tmB, kb * BK, r1, tl.g, full_bar(stage), one);
                 }
@@ -371,8 +398,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         for (int t = unit; ok && t < num_tiles; t += n_units, ++iter) {
             const Tile tl = decode_tile(remap_tile(t, R_t, S_t, C_t), mstart, G, NT, TM, offs);
             const int64_t grow = static_cast<int64_t>(tl.m0) + 128 * static_cast<int>(rank) + row;
-            const bool row_ok = grow < m_cap;
-            const float *sa_row = sA + (row_ok ? grow : 0) * KB;
+            int64_t arow = grow;          // row of A (and sA) this output row is made of
+            if (GATHER) {
+                arow = -1;
+                if (grow < tl.m_end) {
+                    const int v = __ldg(a_map + grow);
+                    if (v >= 0 && v < a_rows) arow = v;
+                }
+            }
+            const bool row_ok = GATHER ? arow >= 0 : grow < m_cap;
+            const float *sa_row = sA + (row_ok ? arow : 0) * KB;
             // scale rows of B for the two column halves of this thread
             int nb0, nb1;
             bool nb1_ok = true;
@@ -571,19 +606,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
 }
 
-// Once per device and tile mode: check the register split and raise the
+// Once per device and kernel variant: check the register split and raise the
 // dynamic shared-memory limit.  Returns a moe_status.
-template <bool PAIR>
+template <bool PAIR, bool GATHER>
 static int prepare_kernel() {
     static int state[MAX_DEVICES] = {};
     static std::mutex mu;
     const int r = once_per_device(state, mu, []() {
         cudaFuncAttributes attr;
-        if (cudaFuncGetAttributes(&attr, grouped_gemm_kernel<PAIR>) != cudaSuccess) return -MOE_ERR_CUDA;
+        if (cudaFuncGetAttributes(&attr, grouped_gemm_kernel<PAIR, GATHER>) != cudaSuccess) return -MOE_ERR_CUDA;
         // setmaxnreg moves registers inside the launch's allotment: the split
         // 128 x 40 + 256 x 232 must equal 384 x (registers at launch)
         if (attr.numRegs != LAUNCH_REGS) return -MOE_ERR_UNSUPPORTED;
-        if (cudaFuncSetAttribute(grouped_gemm_kernel<PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(grouped_gemm_kernel<PAIR, GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(Cfg<PAIR>::SMEM_BYTES)) != cudaSuccess)
             return -MOE_ERR_CUDA;
         return 1;
@@ -608,47 +643,49 @@ static int pair_clusters() {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<true>, &cfg) == cudaSuccess && n > 0) return n;
+        if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<true, false>, &cfg) == cudaSuccess && n > 0)
+            return n;
         return num_sms() / 2;
     });
 }
 
-}  // namespace gg
-}  // namespace moe
-
-using namespace moe;
-
-MOE_API int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets, int64_t m_capacity,
-                                         int64_t N, int64_t K, const uint8_t *A, const float *sA,
-                                         const uint8_t *B, const float *sB, int32_t epilogue, void *C,
-                                         float *sC, int32_t *status, void *stream) {
-    using namespace moe::gg;
+// Both public entry points.  a_map == nullptr: A is [m_capacity, K] in group
+// order (TMA loads); otherwise A is [a_rows, K] and GEMM row m reads A row
+// a_map[m] (gather variant, single tiles).
+static int grouped_gemm(int32_t G, const int32_t *group_offsets, int64_t m_capacity, int64_t N, int64_t K,
+                        const uint8_t *A, const float *sA, const int32_t *a_map, int64_t a_rows, const uint8_t *B,
+                        const float *sB, int32_t epilogue, void *C, float *sC, int32_t *status, void *stream) {
+    const bool gather = a_map != nullptr;
     // tile mode: one-SM tiles unless CTA pairs are asked for (measured on B200:
     // pairs are 25 % slower at 128 tokens per expert, where 256-row tiles are
     // mostly padding, and about 1 % faster at 1024 tokens per expert)
-    const bool single = (epilogue & MOE_GEMM_PAIR_CTA) == 0 || (epilogue & MOE_GEMM_SINGLE_CTA) != 0;
+    const bool single = gather || (epilogue & MOE_GEMM_PAIR_CTA) == 0 || (epilogue & MOE_GEMM_SINGLE_CTA) != 0;
     epilogue &= ~(MOE_GEMM_SINGLE_CTA | MOE_GEMM_PAIR_CTA);
-    if (G < 0 || m_capacity < 0 || N < 0 || K < 0) return MOE_ERR_INVALID_ARG;
+    if (G < 0 || m_capacity < 0 || N < 0 || K < 0 || a_rows < 0) return MOE_ERR_INVALID_ARG;
     if (N % 128 != 0 || K % 128 != 0) return MOE_ERR_INVALID_ARG;
     if (epilogue != MOE_EPI_BF16 && epilogue != MOE_EPI_F32 && epilogue != MOE_EPI_SWIGLU_REQUANT)
         return MOE_ERR_INVALID_ARG;
     if (epilogue == MOE_EPI_SWIGLU_REQUANT && (N % 256 != 0 || !sC)) return MOE_ERR_INVALID_ARG;
     if (G == 0 || m_capacity == 0 || N == 0) return MOE_OK;
     if (K == 0) return MOE_ERR_UNSUPPORTED;   // an empty reduction is not a GEMM this kernel runs
+    if (gather && a_rows == 0) return MOE_ERR_INVALID_ARG;
     const int max_groups = single ? Cfg<false>::MAX_GROUPS : Cfg<true>::MAX_GROUPS;
-    if (G > max_groups || m_capacity > 0x7fffffffLL || N > 0x7fffffffLL || K > 0x7fffffffLL)
+    if (G > max_groups || m_capacity > 0x7fffffffLL || N > 0x7fffffffLL || K > 0x7fffffffLL ||
+        a_rows > 0x7fffffffLL)
         return MOE_ERR_UNSUPPORTED;
     if (!group_offsets || !A || !sA || !B || !sB || !C) return MOE_ERR_INVALID_ARG;
     if (!aligned16(A) || !aligned16(B) || !aligned16(C) || (reinterpret_cast<uintptr_t>(sA) & 3) ||
-        (reinterpret_cast<uintptr_t>(sB) & 3) || (sC && (reinterpret_cast<uintptr_t>(sC) & 3)))
+        (reinterpret_cast<uintptr_t>(sB) & 3) || (sC && (reinterpret_cast<uintptr_t>(sC) & 3)) ||
+        (reinterpret_cast<uintptr_t>(a_map) & 3))
         return MOE_ERR_INVALID_ARG;
-    int rc = single ? prepare_kernel<false>() : prepare_kernel<true>();
+    int rc = gather ? prepare_kernel<false, true>() : single ? prepare_kernel<false, false>()
+                                                              : prepare_kernel<true, false>();
     if (rc != MOE_OK) return rc;
     auto enc = encode_fn();
     if (!enc) return MOE_ERR_CUDA;
 
     CUtensorMap tmA, tmB, tmC;
-    {
+    if (!gather) {
         cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(m_capacity)};
         cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
         cuuint32_t box[2] = {128, 128};
@@ -676,6 +713,17 @@ MOE_API int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets
     // output tiles stored by TMA from the epilogue: bf16 rows in boxes of 32 rows x
     // 64 columns (128-byte swizzle), SwiGLU codes in boxes of 32 rows x 64 columns
     // (64-byte swizzle); the fp32 epilogue stores directly (tmC unused)
+    if (gather) {
+        // source rows of A, gathered four at a time: box one row high
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(a_rows)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+        cuuint32_t box[2] = {128, 1};
+        cuuint32_t es[2] = {1, 1};
+        if (enc(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(A), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MOE_ERR_CUDA;
+    }
     if (epilogue == MOE_EPI_F32) {
         tmC = tmA;
     } else {
@@ -695,9 +743,16 @@ MOE_API int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets
     const int n = static_cast<int>(N), k = static_cast<int>(K);
     const uint64_t wait_ns = wait_limit_ns();
     const int stall = test_stall() ? 1 : 0;
+    if (gather) {
+        grouped_gemm_kernel<false, true><<<num_sms(), THREADS, Cfg<false>::smem_bytes(G), st>>>(
+            tmA, tmB, tmC, group_offsets, G, m_capacity, n, k, sA, sB, epilogue, C, sC, status, wait_ns, stall,
+            a_map, a_rows);
+        return launch_status();
+    }
     if (single) {
-        grouped_gemm_kernel<false><<<num_sms(), THREADS, Cfg<false>::smem_bytes(G), st>>>(
-            tmA, tmB, tmC, group_offsets, G, m_capacity, n, k, sA, sB, epilogue, C, sC, status, wait_ns, stall);
+        grouped_gemm_kernel<false, false><<<num_sms(), THREADS, Cfg<false>::smem_bytes(G), st>>>(
+            tmA, tmB, tmC, group_offsets, G, m_capacity, n, k, sA, sB, epilogue, C, sC, status, wait_ns, stall,
+            nullptr, 0);
         return launch_status();
     }
     cudaLaunchConfig_t cfg = {};
@@ -712,8 +767,32 @@ MOE_API int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<true>, tmA, tmB, tmC, group_offsets, G, m_capacity, n, k, sA, sB,
-                           static_cast<int>(epilogue), C, sC, status, wait_ns, 0) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<true, false>, tmA, tmB, tmC, group_offsets, G, m_capacity, n, k,
+                           sA, sB, static_cast<int>(epilogue), C, sC, status, wait_ns, 0,
+                           static_cast<const int32_t *>(nullptr), static_cast<int64_t>(0)) != cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_status();
+}
+
+}  // namespace gg
+}  // namespace moe
+
+using namespace moe;
+
+MOE_API int fp8_grouped_gemm_blockscaled(int32_t G, const int32_t *group_offsets, int64_t m_capacity,
+                                         int64_t N, int64_t K, const uint8_t *A, const float *sA,
+                                         const uint8_t *B, const float *sB, int32_t epilogue, void *C,
+                                         float *sC, int32_t *status, void *stream) {
+    return gg::grouped_gemm(G, group_offsets, m_capacity, N, K, A, sA, nullptr, 0, B, sB, epilogue, C, sC, status,
+                            stream);
+}
+
+MOE_API int fp8_grouped_gemm_blockscaled_gather(int32_t G, const int32_t *group_offsets, int64_t m_capacity,
+                                                int64_t N, int64_t K, const uint8_t *A, const float *sA,
+                                                int64_t a_rows, const int32_t *a_map, const uint8_t *B,
+                                                const float *sB, int32_t epilogue, void *C, float *sC,
+                                                int32_t *status, void *stream) {
+    if (!a_map) return MOE_ERR_INVALID_ARG;
+    return gg::grouped_gemm(G, group_offsets, m_capacity, N, K, A, sA, a_map, a_rows, B, sB, epilogue, C, sC, status,
+                            stream);
 }

@@ -95,6 +95,20 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *tm,
         : "memory");
 }
 
+// TMA gather of four rows: rows y0..y3 of a 2D tensor map whose box is one row
+// high, columns x .. x + box - 1 (x * element size a multiple of 16 bytes),
+// landing at dst as four consecutive box rows in the map's swizzle, which is a
+// function of the shared-memory address (so four rows at dst = atom + 512 take
+// rows 4..7 of a 1024-byte 128B-swizzle atom).  Issued by the calling thread.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *tm, int32_t x, int32_t y0, int32_t y1,
+                                            int32_t y2, int32_t y3, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar)
+        : "memory");
+}
+
 // Plain (untiled) bulk copy global -> this CTA's shared memory, completing on
 // an mbarrier; both addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,

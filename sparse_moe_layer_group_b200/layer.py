@@ -12,7 +12,13 @@ the forward runs in the library's kernels:
                       into the first T*K rows
   4  grouped GEMM     W13 of the E routed experts and, as group E, of the
                       shared expert over the T token rows; SwiGLU + 1x128
-                      requant fused
+                      requant fused.  With gather=True the permute writes only
+                      the maps (3 kernels) and the GEMM fetches each routed row
+                      from the token's quantised row through tok_of with TMA
+                      row gathers, so the permuted copy is never written; same
+                      bits, but measured slower on B200 at the DeepSeek-V3
+                      shape (32 four-row gathers per A tile instead of one
+                      tiled load), hence not the default
   5  grouped GEMM     W2 of the same E + 1 groups -> bf16 rows
   6  moe_combine      gate-weighted sum of the K rows + the shared row -> bf16
   (7 moe_bias_update  after the step, from the expert loads of step 3)
@@ -31,7 +37,7 @@ import torch
 
 from . import _abi as abi
 
-LAUNCHES_PER_FORWARD = 10   # 2 route + 1 quant + 4 permute + 2 GEMM + 1 combine
+LAUNCHES_PER_FORWARD = 10   # 2 route + 1 quant + 4 permute + 2 GEMM + 1 combine (gather=True: 9)
 
 
 @dataclass
@@ -83,8 +89,10 @@ class MoELayer:
 
     def __init__(self, T: int, H: int, E: int, K: int, n_group: int, topk_group: int, I: int,
                  rho: float, w_router: torch.Tensor, e_bias: torch.Tensor, weights: QuantWeights,
-                 router_offset: Optional[torch.Tensor] = None, device="cuda"):
+                 router_offset: Optional[torch.Tensor] = None, device="cuda", gather: bool = False):
         self.T, self.H, self.E, self.K, self.I = T, H, E, K, I
+        self.gather = gather
+        self.launches_per_forward = LAUNCHES_PER_FORWARD - (1 if gather else 0)
         self.n_group, self.topk_group, self.rho = n_group, topk_group, rho
         self.d = abi.dims(T, H, E, K, n_group, topk_group, I, rho)
         self.w_router, self.e_bias, self.router_offset = w_router, e_bias, router_offset
@@ -105,18 +113,29 @@ class MoELayer:
         self.scores = torch.empty(T, E, **f32)
         ws_bytes = max(abi.workspace_size(self.d), 256)
         self.ws = torch.empty((ws_bytes + 255) // 256 * 256, **u8)
-        # A of both GEMM launches: rows 0..T*K-1 the routed (token, slot) pairs
-        # in expert order, rows T*K..T*K+T-1 the tokens themselves (shared expert)
-        self.aq = torch.empty(TK + T, H, **u8)
-        self.as_ = torch.empty(TK + T, H // 128, **f32)
-        self.xq = self.aq[TK:]
-        self.xs = self.as_[TK:]
+        # rows of the first GEMM: rows 0..T*K-1 the routed (token, slot) pairs in
+        # expert order, rows T*K..T*K+T-1 the tokens themselves (shared expert)
+        if gather:
+            # read through a_map = (tok_of, 0..T-1) from the T quantised token rows
+            self.aq = self.as_ = None
+            self.xq = torch.empty(T, H, **u8)
+            self.xs = torch.empty(T, H // 128, **f32)
+            self.a_map = torch.empty(TK + T, **i32)
+            self.a_map[TK:] = torch.arange(T, **i32)
+            self.tok_of = self.a_map[:TK]
+        else:
+            # a materialised copy in that order; the last T rows are the quantiser's output
+            self.aq = torch.empty(TK + T, H, **u8)
+            self.as_ = torch.empty(TK + T, H // 128, **f32)
+            self.xq = self.aq[TK:]
+            self.xs = self.as_[TK:]
+            self.a_map = None
+            self.tok_of = torch.empty(TK, **i32)
         self.load = torch.empty(E, **i32)
         # group offsets of the E + 1 groups: moe_permute writes entries 0..E,
         # entry E + 1 closes the shared group
         self.offsets_all = torch.full((E + 2,), TK + T, **i32)
         self.offsets = self.offsets_all[:E + 1]
-        self.tok_of = torch.empty(TK, **i32)
         self.row_of = torch.empty(TK, **i32)
         self.actq = torch.empty(TK + T, I, **u8)
         self.acts = torch.empty(TK + T, I // 128, **f32)
@@ -150,14 +169,23 @@ class MoELayer:
         abi.moe_route_pieces(self.d, x, self.w_pieces, self.e_bias, self.router_offset, self.topk_idx,
                              self.topk_w, self.scores, self.ws, st, stream)
         abi.fp8_quant_1x128(x, self.xq, self.xs, st, stream)
-        abi.moe_permute(self.d, self.topk_idx, self.xq, self.xs, self.load, self.offsets, self.tok_of,
-                        self.row_of, self.aq, self.as_, self.ws, st, stream)
+        if self.gather:
+            abi.moe_permute(self.d, self.topk_idx, None, None, self.load, self.offsets, self.tok_of,
+                            self.row_of, None, None, self.ws, st, stream)
+        else:
+            abi.moe_permute(self.d, self.topk_idx, self.xq, self.xs, self.load, self.offsets, self.tok_of,
+                            self.row_of, self.aq, self.as_, self.ws, st, stream)
         qw = self.qw
         ev_stream = torch.cuda.current_stream() if stream is None else stream
         if gemm_events is not None:
             gemm_events[0].record(ev_stream)
-        abi.fp8_grouped_gemm_blockscaled(E + 1, self.offsets_all, M, 2 * I, H, self.aq, self.as_, qw.w13, qw.s13,
-                                         abi.MOE_EPI_SWIGLU_REQUANT, self.actq, self.acts, st, stream)
+        if self.gather:
+            abi.fp8_grouped_gemm_blockscaled_gather(E + 1, self.offsets_all, M, 2 * I, H, self.xq, self.xs,
+                                                    self.a_map, qw.w13, qw.s13, abi.MOE_EPI_SWIGLU_REQUANT,
+                                                    self.actq, self.acts, st, stream)
+        else:
+            abi.fp8_grouped_gemm_blockscaled(E + 1, self.offsets_all, M, 2 * I, H, self.aq, self.as_, qw.w13,
+                                             qw.s13, abi.MOE_EPI_SWIGLU_REQUANT, self.actq, self.acts, st, stream)
         if gemm_events is not None:
             gemm_events[1].record(ev_stream)
         abi.fp8_grouped_gemm_blockscaled(E + 1, self.offsets_all, M, H, I, self.actq, self.acts, qw.w2, qw.s2,

@@ -76,6 +76,14 @@ def test_host_validation_rejects_before_launch():
     for mode in (0, a.MOE_GEMM_PAIR_CTA):
         assert L.fp8_grouped_gemm_blockscaled(4001, 16, 64, 256, 128, 16, 16, 16, 16, mode, 16, None, None,
                                               None) == a.MOE_ERR_UNSUPPORTED
+    # gather variant: the row map is required and 4-byte aligned, a_rows >= 1
+    gg = L.fp8_grouped_gemm_blockscaled_gather
+    assert gg(1, 16, 64, 256, 128, 16, 16, 8, None, 16, 16, 0, 16, None, None, None) == a.MOE_ERR_INVALID_ARG
+    assert gg(1, 16, 64, 256, 128, 16, 16, 8, 18, 16, 16, 0, 16, None, None, None) == a.MOE_ERR_INVALID_ARG
+    assert gg(1, 16, 64, 256, 128, 16, 16, -1, 16, 16, 16, 0, 16, None, None, None) == a.MOE_ERR_INVALID_ARG
+    assert gg(1, 16, 64, 256, 128, 16, 16, 0, 16, 16, 16, 0, 16, None, None, None) == a.MOE_ERR_INVALID_ARG
+    assert gg(1, 16, 64, 256, 100, 16, 16, 8, 16, 16, 16, 0, 16, None, None, None) == a.MOE_ERR_INVALID_ARG
+    assert gg(0, 16, 64, 256, 128, 16, 16, 8, 16, 16, 16, 0, 16, None, None, None) == 0
     # zero-size work is a no-op
     assert L.fp8_grouped_gemm_blockscaled(0, 16, 64, 256, 128, 16, 16, 16, 16, 0, 16, None, None, None) == 0
     assert L.fp8_quant_1x128(16, 0, 128, 16, 16, None, None) == 0

@@ -16,7 +16,7 @@ from tests.test_gpu_kernels import check_routing, routing_tol
 pytestmark = pytest.mark.gpu
 
 
-def build_layer(lib, shape, device="cuda", T=None, offset=None):
+def build_layer(lib, shape, device="cuda", T=None, offset=None, gather=False):
     """Layer with synth weights drawn on `device` (per expert, regenerable)."""
     T = shape.T if T is None else T
     H, E, I = shape.H, shape.E, shape.I
@@ -31,7 +31,7 @@ def build_layer(lib, shape, device="cuda", T=None, offset=None):
     b = synth.expert_bias(E, shape.bias_range, synth.seed_of(shape, synth.BIAS), device=device)
     layer = lib.MoELayer(T, H, E, shape.K, shape.n_group, shape.topk_group, I, shape.rho,
                          wr.cuda().contiguous(), b.cuda().contiguous(), qw,
-                         router_offset=None if offset is None else offset.cuda())
+                         router_offset=None if offset is None else offset.cuda(), gather=gather)
     return layer, master, wr, b
 
 
@@ -189,3 +189,24 @@ def test_layer_caller_owned_output(lib):
     assert torch.equal(buf, ref)
     with pytest.raises(ValueError):
         layer.forward(x, out=torch.empty(shape.T, shape.H, dtype=torch.float32, device="cuda"))
+
+
+@pytest.mark.parametrize("shape", [synth.TINY, synth.MID, pytest.param(synth.DSV3, marks=pytest.mark.slow)])
+def test_layer_gather_equals_materialised(lib, shape):
+    """The forward whose W13 gathers its A rows through tok_of and the default
+    forward over the materialised permuted copy give the same bits at every
+    stage: the gather changes where the GEMM reads a row, not its arithmetic."""
+    dev = "cuda" if shape is synth.DSV3 else "cpu"
+    lay_g, master, wr, b = build_layer(lib, shape, device=dev, gather=True)
+    lay_m = lib.MoELayer(shape.T, shape.H, shape.E, shape.K, shape.n_group, shape.topk_group, shape.I, shape.rho,
+                         lay_g.w_router, b.cuda().contiguous(), lay_g.qw, gather=False)
+    assert lay_g.aq is None and lay_m.aq is not None
+    x = synth.activations(shape.T, shape.H, synth.seed_of(shape, synth.X), shape.x_outlier_frac, device=dev)
+    x = cuda(x)
+    og = lay_g.forward(x).clone()
+    om = lay_m.forward(x).clone()
+    torch.cuda.synchronize()
+    assert int(lay_g.status.item()) == 0 and int(lay_m.status.item()) == 0
+    for name in ("topk_idx", "load", "offsets", "tok_of", "row_of", "xq", "xs", "actq", "acts", "yperm"):
+        assert torch.equal(getattr(lay_g, name), getattr(lay_m, name)), name
+    assert torch.equal(og, om)
