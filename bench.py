@@ -548,15 +548,17 @@ def leg_wgrad(offsets_all, pk, iters: int = 5) -> dict:
 
     step()
     torch.cuda.synchronize()
+    time.sleep(0.5)              # after the prefill and decode legs: let the clocks recover
     evs = []
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(iters):
-        ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-        evs.append(ev)
-        step(ev)
-    t1.record()
-    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0.record()
+        for _ in range(iters):
+            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            evs.append(ev)
+            step(ev)
+        t1.record()
+        torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / iters
     g_ms = statistics.median(a.elapsed_time(b) for a, b in evs)
     flops = 2.0 * M * 2 * I * H
@@ -570,7 +572,7 @@ def leg_wgrad(offsets_all, pk, iters: int = 5) -> dict:
             "gemm_ms": round(g_ms, 4), "gemm_tflops": round(flops / g_ms / 1e9, 1),
             "gemm_gbs": round((out_bytes + in_bytes) / g_ms / 1e6, 1),
             "gemm_frac_of_hbm": round((out_bytes + in_bytes) / g_ms / 1e6 / pk["hbm_gbs"], 3),
-            "algorithmic_bytes": out_bytes + in_bytes, "device_status": status}
+            "algorithmic_bytes": out_bytes + in_bytes, "device_status": status, "clocks": clk.summary()}
 
 
 def leg_gather(layer, pk, iters: int = 10) -> dict:

@@ -100,18 +100,20 @@ __device__ __forceinline__ float swiglu_act(float g, float u) {
 //
 // q = fp32(v * inv) differs from v / s by at most 2^-24 |v/s| (the reciprocal)
 // plus half an ulp (the product), so the correctly rounded quotient lies
-// within three steps of the fp32 grid from q, on q's side of zero.  E4M3
-// rounding is monotone in the magnitude, so when |q| lowered and raised by four
-// grid steps gives the same code, that code is the quotient's; otherwise (a
-// quotient within a few fp32 ulps of an E4M3 rounding boundary, or a reciprocal
-// that overflowed) the quotient is computed by the correctly rounded division.
+// within three steps of the fp32 grid from q, on q's side of zero.  For |q| in
+// the E4M3 normal range (>= 2^-6) the E4M3 rounding boundaries of q's binade
+// are the fp32 values whose 20 bits below E4M3's three mantissa bits read
+// 0x80000 (binade edges are E4M3 values), and E4M3 rounding is monotone; so
+// when those 20 bits of q are more than four steps from 0x80000, the quotient
+// rounds to q's code.  Otherwise (a quotient within a few fp32 ulps of a
+// boundary, |q| below 2^-6 where E4M3 is subnormal, or a reciprocal that
+// overflowed) the quotient is computed by the correctly rounded division.
 __device__ __forceinline__ uint32_t e4m3x2_cvt(float a, float b) {
     return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
 }
-__device__ __forceinline__ float grid_steps(float q, int n) {   // |q| moved by n fp32 steps, sign kept
-    const uint32_t u = __float_as_uint(q), sgn = u & 0x80000000u;
-    const int m = static_cast<int>(u ^ sgn) + n;   // |q| < 2^31 as a bit pattern
-    return __uint_as_float(sgn | static_cast<uint32_t>(m < 0 ? 0 : m));
+__device__ __forceinline__ bool e4m3_near_boundary(float q) {
+    const uint32_t u = __float_as_uint(q) & 0x7fffffffu;
+    return (u != 0u && u < 0x3C800000u) || ((u & 0xFFFFFu) - 0x7FFFCu) <= 8u;
 }
 // E4M3 codes of fp32(a * inv) and fp32(b * inv), inv the correctly rounded
 // reciprocal of the tile scale: the fast form of the requantisation, within 1.5
@@ -122,9 +124,7 @@ __device__ __forceinline__ uint32_t e4m3x2_rcp(float a, float b, float inv) {
 __device__ __forceinline__ uint32_t e4m3x2_div(float a, float b, float s, float inv) {
     if (isfinite(inv)) {
         const float qa = __fmul_rn(a, inv), qb = __fmul_rn(b, inv);
-        const uint32_t lo = e4m3x2_cvt(grid_steps(qa, -4), grid_steps(qb, -4));
-        const uint32_t hi = e4m3x2_cvt(grid_steps(qa, 4), grid_steps(qb, 4));
-        if (lo == hi) return lo;
+        if (!e4m3_near_boundary(qa) && !e4m3_near_boundary(qb)) return e4m3x2_cvt(qa, qb);
     }
     return e4m3x2_cvt(__fdiv_rn(a, s), __fdiv_rn(b, s));
 }

@@ -6,73 +6,80 @@
 // the granularities of the "From technical report to a runnable config" guide
 // (lpnh.cn), section 3: inputs tile-wise 1x128, weights block-wise 128x128, e4m3.
 //
-// All three kernels are HBM-bound streams: 16-byte vector loads, one warp half
-// (16 lanes x 8 values) per 1x128 tile, shuffles for the tile amax.
+// All three kernels are HBM-bound streams: 16-byte vector loads, a group of
+// lanes per tile, shuffles for the tile amax.
 #include "common.cuh"
 
 namespace moe {
 
-// 16 lanes own one 1x128 tile: lane l holds columns 8l .. 8l+7.  Each trip
-// handles Q tiles per half-warp with all Q loads issued first, so several
-// 16-byte loads per thread are in flight.
+// 8 lanes own one 1x128 tile: lane l holds columns 16l .. 16l+15 (two 16-byte
+// loads, one 16-byte store of codes).  Each trip handles Q tiles per 8-lane
+// group with all loads issued first, so several loads per thread are in flight.
 template <int Q>
-__device__ __forceinline__ void quant_tiles(const uint4 *__restrict__ x, uint2 *__restrict__ q,
+__device__ __forceinline__ void quant_tiles(const uint4 *__restrict__ x, uint4 *__restrict__ q,
                                             float *__restrict__ scales, int64_t first, int64_t stride,
-                                            int64_t n_tiles, int lane16, int32_t *status) {
-    uint4 v[Q];
+                                            int64_t n_tiles, int lane8, int32_t *status) {
+    uint4 v[Q][2];
 #pragma unroll
     for (int u = 0; u < Q; ++u) {
         const int64_t tile = first + u * stride;
-        v[u] = tile < n_tiles ? __ldg(x + tile * 16 + lane16) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            v[u][h] = tile < n_tiles ? __ldg(x + tile * 16 + lane8 * 2 + h) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int u = 0; u < Q; ++u) {
         const int64_t tile = first + u * stride;
-        const float f[8] = {bf16_lo(v[u].x), bf16_hi(v[u].x), bf16_lo(v[u].y), bf16_hi(v[u].y),
-                            bf16_lo(v[u].z), bf16_hi(v[u].z), bf16_lo(v[u].w), bf16_hi(v[u].w)};
-        float amax = 0.0f;
-        bool fin = true;
+        float f[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) amax_step(f[i], amax, fin);
-        int fin_i = fin ? 1 : 0;
-#pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) {
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            fin_i &= __shfl_xor_sync(0xffffffffu, fin_i, o);
+        for (int h = 0; h < 2; ++h) {
+            f[8 * h + 0] = bf16_lo(v[u][h].x); f[8 * h + 1] = bf16_hi(v[u][h].x);
+            f[8 * h + 2] = bf16_lo(v[u][h].y); f[8 * h + 3] = bf16_hi(v[u][h].y);
+            f[8 * h + 4] = bf16_lo(v[u][h].z); f[8 * h + 5] = bf16_hi(v[u][h].z);
+            f[8 * h + 6] = bf16_lo(v[u][h].w); f[8 * h + 7] = bf16_hi(v[u][h].w);
         }
+        // max |v| as the max of the magnitude bit patterns (ordered like the
+        // values); a pattern >= 0x7f800000 is an Inf or NaN in the tile
+        uint32_t um[2] = {0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 16; ++i) um[i & 1] = max(um[i & 1], __float_as_uint(f[i]) & 0x7fffffffu);
+        uint32_t umax = max(um[0], um[1]);
+#pragma unroll
+        for (int o = 4; o >= 1; o >>= 1) umax = max(umax, __shfl_xor_sync(0xffffffffu, umax, o));
         if (tile >= n_tiles) continue;
-        const bool finite = fin_i != 0;
-        const float sc = tile_scale(amax, finite);
+        const bool finite = umax < 0x7f800000u;
+        const float sc = tile_scale(__uint_as_float(umax), finite);
         // codes of the correctly rounded quotients v / scale, two at a time
-        // (e4m3x2_div: the product with the reciprocal, confirmed or replaced by
-        // the division wherever it could straddle an E4M3 rounding boundary)
+        // (e4m3x2_div: the product with the reciprocal wherever it provably
+        // rounds like the quotient, else the division)
         const float inv = __frcp_rn(sc);
-        const uint32_t lo = finite ? e4m3x2_div(f[0], f[1], sc, inv) | e4m3x2_div(f[2], f[3], sc, inv) << 16
-                                   : 0x7F7F7F7Fu;
-        const uint32_t hi = finite ? e4m3x2_div(f[4], f[5], sc, inv) | e4m3x2_div(f[6], f[7], sc, inv) << 16
-                                   : 0x7F7F7F7Fu;
-        q[tile * 16 + lane16] = make_uint2(lo, hi);
-        if (lane16 == 0) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            w[i] = finite ? e4m3x2_div(f[4 * i], f[4 * i + 1], sc, inv) | e4m3x2_div(f[4 * i + 2], f[4 * i + 3], sc, inv) << 16
+                          : 0x7F7F7F7Fu;
+        q[tile * 8 + lane8] = make_uint4(w[0], w[1], w[2], w[3]);
+        if (lane8 == 0) {
             scales[tile] = sc;
             if (!finite) set_flag(status, MOE_FLAG_NONFINITE);
         }
     }
 }
 
-constexpr int QUANT_Q = 4;
+constexpr int QUANT_Q = 2;
 
 __global__ void __launch_bounds__(256) quant_1x128_kernel(const uint4 *__restrict__ x,
-                                                          uint2 *__restrict__ q,
+                                                          uint4 *__restrict__ q,
                                                           float *__restrict__ scales,
                                                           int64_t n_tiles, int32_t *status) {
-    const int lane16 = threadIdx.x & 15;
-    const int64_t half_id = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
-    const int64_t n_halves = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 4;
-    // every 16-lane half runs the same trip count so the shuffles stay converged
-    const int64_t per_trip = n_halves * QUANT_Q;
+    const int lane8 = threadIdx.x & 7;
+    const int64_t group = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 3;
+    const int64_t n_groups = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 3;
+    // every 8-lane group runs the same trip count so the shuffles stay converged
+    const int64_t per_trip = n_groups * QUANT_Q;
     const int64_t trips = (n_tiles + per_trip - 1) / per_trip;
     for (int64_t it = 0; it < trips; ++it)
-        quant_tiles<QUANT_Q>(x, q, scales, half_id + it * per_trip, n_halves, n_tiles, lane16, status);
+        quant_tiles<QUANT_Q>(x, q, scales, group + it * per_trip, n_groups, n_tiles, lane8, status);
 }
 
 // One CTA per 128x128 block: 256 threads, each row of the block is 16 lanes x 16 B.
@@ -184,12 +191,15 @@ MOE_API int fp8_quant_1x128(const void *x, int64_t rows, int64_t cols, uint8_t *
     if (!x || !q || !scales || !aligned16(x) || !aligned16(q) || !aligned16(scales))
         return MOE_ERR_INVALID_ARG;
     const int64_t n_tiles = rows * (cols / 128);
-    const int64_t tiles_per_block = 256 / 16 * QUANT_Q;
+    // one trip per half-warp up to a million blocks (the hardware schedules the
+    // blocks as SMs free up, so no trip is left mostly idle); beyond that the
+    // half-warps loop over further trips
+    const int64_t tiles_per_block = 256 / 8 * QUANT_Q;
     int64_t blocks = (n_tiles + tiles_per_block - 1) / tiles_per_block;
-    const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+    const int64_t cap = int64_t(1) << 20;
     if (blocks > cap) blocks = cap;
     quant_1x128_kernel<<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(
-        reinterpret_cast<const uint4 *>(x), reinterpret_cast<uint2 *>(q), scales, n_tiles, status);
+        reinterpret_cast<const uint4 *>(x), reinterpret_cast<uint4 *>(q), scales, n_tiles, status);
     return launch_status();
 }
 

@@ -13,7 +13,8 @@
 //   router_split_kernel / router_tc_kernel (router_tc.cu)  fp32-exact logits on
 //                         the tensor cores, split over K into partial sums.
 //   route_select_kernel   one warp per token: adds the partial logits in split
-//                         order, offset, sigmoid; group scores, group pick, top-K,
+//                         order, offset, sigmoid; group scores, group pick, top-K
+//                         (warp max/min reductions over order-preserving keys),
 //                         gates in float64 (exact sum of <= 32 fp32 values).
 #include <cfloat>
 
@@ -21,118 +22,158 @@
 
 namespace moe {
 
-// (value, index) order used for every ranking: larger value first, then the
-// lower index.
-__device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
-    return v > bv || (v == bv && i < bi);
-}
-
-__device__ __forceinline__ void warp_best(float &v, int &i) {
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, v, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, i, o);
-        if (better(ov, oi, v, i)) { v = ov; i = oi; }
-    }
-}
-
 constexpr int SEL_WARPS = 8;
 constexpr int SEL_MAX_E = 1024;
 
-// One warp per token.  The affinities come either given (s_in [T, E]) or as
-// n_split fp32 partial logits [n_split, T, E] from the tensor-core router, which
-// are added in split order (a fixed order, so results are deterministic), offset
-// and passed through the sigmoid here.  r = s + b is formed where it is used.
+// Order-preserving map of an fp32 value to uint32 (larger value -> larger
+// key); NaN maps below every number, so it is never preferred.
+__device__ __forceinline__ uint32_t order_key(float v) {
+    const uint32_t u = __float_as_uint(v);
+    if (v != v) return 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Best (largest value, then lowest index) of one candidate per lane, by two
+// warp reductions: the largest key, then the lowest index holding it.
+__device__ __forceinline__ int warp_best_index(float v, int i) {
+    const uint32_t k = order_key(v);
+    const uint32_t mx = __reduce_max_sync(0xffffffffu, k);
+    return static_cast<int>(__reduce_min_sync(0xffffffffu, k == mx ? static_cast<uint32_t>(i) : 0xffffffffu));
+}
+
+// One warp per token; lane l holds experts l + 32 j, j < PER (PER >= ceil(E/32)).
+// The affinities come either given (s_in [T, E]) or as n_split fp32 partial
+// logits [n_split, T, E] from the tensor-core router, which are added in split
+// order (a fixed order, so results are deterministic), offset and passed through
+// the sigmoid here.  r = s + b is kept in registers; every ranking orders by
+// value, then by the lower index.
+template <int PER>
 __global__ void __launch_bounds__(SEL_WARPS * 32) route_select_kernel(
     const float *__restrict__ s_in, const float *__restrict__ partial, int n_split,
     const float *__restrict__ offset, float *__restrict__ s_out, const float *__restrict__ bias,
     int32_t *__restrict__ topk_idx, float *__restrict__ topk_w, int T, int E, int K, int n_group,
     int topk_group, float rho) {
-    extern __shared__ float sh[];   // SEL_WARPS * E affinities
+    extern __shared__ float sh[];   // SEL_WARPS * 2 * E: affinities s, then r = s + b
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int t = blockIdx.x * SEL_WARPS + wid;
     if (t >= T) return;
-    float *srow = sh + wid * E;
+    float *srow = sh + wid * 2 * E;
+    float *rrow = srow + E;
+    float r[PER];
     if (partial) {
         const int64_t plane = static_cast<int64_t>(T) * E;
         const float *base = partial + static_cast<int64_t>(t) * E;
-        // eight experts per lane at a time: the eight loads of one split are
-        // independent, so a split costs one memory round trip; every logit is
-        // still summed in split order
-        for (int e0 = 0; e0 < E; e0 += 256) {
-            float l[8];
+        float l[PER];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int e = e0 + lane + 32 * j;
-                l[j] = e < E ? base[e] : 0.0f;
-            }
-#pragma unroll 4
-            for (int q = 1; q < n_split; ++q) {
-                const float *pq = base + q * plane;
-                float v[8];
+        for (int j = 0; j < PER; ++j) {
+            const int e = lane + 32 * j;
+            l[j] = e < E ? base[e] : 0.0f;
+        }
+        // four splits' loads in flight at a time; each logit still sums in split order
+        int q = 1;
+        for (; q + 3 < n_split; q += 4) {
+            float v[4][PER];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int e = e0 + lane + 32 * j;
-                    v[j] = e < E ? pq[e] : 0.0f;
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int j = 0; j < PER; ++j) {
+                    const int e = lane + 32 * j;
+                    v[u][j] = e < E ? base[(q + u) * plane + e] : 0.0f;
                 }
 #pragma unroll
-                for (int j = 0; j < 8; ++j) l[j] = __fadd_rn(l[j], v[j]);
-            }
+            for (int u = 0; u < 4; ++u)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int e = e0 + lane + 32 * j;
-                if (e < E) {
-                    const float lj = offset ? __fadd_rn(l[j], __ldg(offset + e)) : l[j];
-                    const float sv = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-lj)));
-                    srow[e] = sv;
-                    if (s_out) s_out[static_cast<int64_t>(t) * E + e] = sv;
-                }
+                for (int j = 0; j < PER; ++j) l[j] = __fadd_rn(l[j], v[u][j]);
+        }
+        for (; q < n_split; ++q) {
+#pragma unroll
+            for (int j = 0; j < PER; ++j) {
+                const int e = lane + 32 * j;
+                l[j] = __fadd_rn(l[j], e < E ? base[q * plane + e] : 0.0f);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E) {
+                const float lj = offset ? __fadd_rn(l[j], __ldg(offset + e)) : l[j];
+                const float sv = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-lj)));
+                srow[e] = sv;
+                if (s_out) s_out[static_cast<int64_t>(t) * E + e] = sv;
+                r[j] = __fadd_rn(sv, __ldg(bias + e));
+                rrow[e] = r[j];
+            } else {
+                r[j] = -INFINITY;
             }
         }
     } else {
-        for (int e = lane; e < E; e += 32) srow[e] = s_in[static_cast<int64_t>(t) * E + e];
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E) {
+                const float sv = s_in[static_cast<int64_t>(t) * E + e];
+                srow[e] = sv;
+                r[j] = __fadd_rn(sv, __ldg(bias + e));
+                rrow[e] = r[j];
+            } else {
+                r[j] = -INFINITY;
+            }
+        }
     }
     __syncwarp();
     const int gs = E / n_group;
-    // group scores: lane g scans its group for the two largest values of r
+    // group scores: lane g takes the two largest r of its group (a repeated
+    // maximum counts twice) from shared memory
     float gscore = -FLT_MAX;
     const bool gvalid = lane < n_group;
     if (gvalid) {
         float m1 = -FLT_MAX, m2 = -FLT_MAX;
+        const float *gr = rrow + lane * gs;
+#pragma unroll 8
         for (int j = 0; j < gs; ++j) {
-            const int e = lane * gs + j;
-            const float v = __fadd_rn(srow[e], __ldg(bias + e));
+            const float v = gr[j];
             if (v > m1) { m2 = m1; m1 = v; } else if (v > m2) { m2 = v; }
         }
         gscore = gs == 1 ? m1 : __fadd_rn(m1, m2);
     }
-    // keep the topk_group best groups (ties to the lower group)
-    uint32_t kept = 0;
-    bool taken_g = !gvalid;
-    for (int round = 0; round < topk_group; ++round) {
-        float v = taken_g ? -INFINITY : gscore;
-        int i = taken_g ? 0x7fffffff : lane;
-        warp_best(v, i);
-        kept |= 1u << i;
-        if (lane == i) taken_g = true;
+    // keep the topk_group best groups (ties to the lower group): a group's rank
+    // is the number of groups ahead of it
+    int rank = 0;
+    for (int h = 0; h < n_group; ++h) {
+        const float o = __shfl_sync(0xffffffffu, gscore, h);
+        rank += (o > gscore || (o == gscore && h < lane)) ? 1 : 0;
     }
-    // top-K over the kept groups' experts
-    uint32_t taken = 0;   // bit j: expert lane + 32 j already chosen (E <= 1024)
+    const uint32_t kept = __ballot_sync(0xffffffffu, gvalid && rank < topk_group);
+    // top-K over the kept groups' experts: each lane keeps its own best
+    // candidate; per round the warp's best is taken and only its lane rescans
+    uint32_t taken = 0;   // bit j: expert lane + 32 j chosen, or not selectable
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+        const int e = lane + 32 * j;
+        if (e >= E || !(kept >> (e / gs) & 1u)) taken |= 1u << j;
+    }
+    auto local_best = [&](float &bv, int &bi) {
+        bv = -INFINITY;
+        bi = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const float v = r[j];
+            const int e = lane + 32 * j;
+            if (!(taken >> j & 1u) && (v > bv || (v == bv && e < bi) || bi == 0x7fffffff)) { bv = v; bi = e; }
+        }
+    };
+    float bv;
+    int bi;
+    local_best(bv, bi);
     float my_s = 0.0f;
     int my_i = -1;
-    const int per_lane = (E + 31) / 32;
     for (int k = 0; k < K; ++k) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
-        for (int j = 0; j < per_lane; ++j) {
-            const int e = lane + 32 * j;
-            if (e >= E || (taken >> j & 1u) || !(kept >> (e / gs) & 1u)) continue;
-            const float v = __fadd_rn(srow[e], __ldg(bias + e));
-            if (better(v, e, bv, bi)) { bv = v; bi = e; }
+        const int w = warp_best_index(bv, bi);
+        if ((w & 31) == lane) {
+            taken |= 1u << (w >> 5);
+            local_best(bv, bi);
         }
-        warp_best(bv, bi);
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        if (lane == k) { my_i = bi; my_s = srow[bi]; }
+        if (lane == k) { my_i = w; my_s = srow[w]; }
     }
     // gates: (rho * s_k) / sum s_j in float64 (the sum of <= 32 fp32 values in (0,1) is exact)
     double sum = lane < K ? static_cast<double>(my_s) : 0.0;
@@ -159,11 +200,23 @@ static int launch_select(const moe_dims *d, const float *s_in, const float *part
                          const float *offset, float *s_out, const float *e_bias, int32_t *idx, float *w,
                          cudaStream_t st) {
     const int blocks = (d->T + SEL_WARPS - 1) / SEL_WARPS;
-    const size_t smem = static_cast<size_t>(SEL_WARPS) * d->E * sizeof(float);
-    route_select_kernel<<<blocks, SEL_WARPS * 32, smem, st>>>(s_in, partial, n_split, offset, s_out, e_bias, idx,
-                                                              w, d->T, d->E, d->K, d->n_group, d->topk_group,
-                                                              d->routed_scaling_factor);
-    return launch_status();
+    const size_t smem = static_cast<size_t>(SEL_WARPS) * 2 * d->E * sizeof(float);
+    const int per = (d->E + 31) / 32;
+    auto go = [&](auto kern) -> int {
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+                cudaSuccess)
+            return MOE_ERR_CUDA;
+        kern<<<blocks, SEL_WARPS * 32, smem, st>>>(s_in, partial, n_split, offset, s_out, e_bias, idx, w, d->T, d->E,
+                                                   d->K, d->n_group, d->topk_group, d->routed_scaling_factor);
+        return launch_status();
+    };
+    if (per <= 1) return go(route_select_kernel<1>);
+    if (per <= 2) return go(route_select_kernel<2>);
+    if (per <= 4) return go(route_select_kernel<4>);
+    if (per <= 8) return go(route_select_kernel<8>);
+    if (per <= 16) return go(route_select_kernel<16>);
+    return go(route_select_kernel<32>);
 }
 
 int router_splits(int T, int E, int H);
