@@ -25,7 +25,14 @@ tokens).  One forward on each rank:
 
 Every arithmetic step runs in the library's kernels (or, in the CPU tests, in
 an injected stand-in of the binding); torch.distributed only moves buffers.
-The bias update from the global expert loads is not part of this class.
+
+The bias update (section 3.3 of the walkthrough: b_e moves by gamma against the
+imbalance of expert e's load over the batch) needs every expert's load over all
+ranks' tokens.  Expert e's global load is exactly the number of rows rank
+e % world received for it (the local permutation's load), so bias_update
+all-gathers the local loads into the global vector and every rank applies the
+same update to its copy of the bias: the copies stay identical without
+exchanging the bias itself.
 """
 from __future__ import annotations
 
@@ -88,7 +95,8 @@ class EPMoELayer:
         self.recv_q = torch.empty(Rmax, H, **u8)
         self.recv_s = torch.empty(Rmax, H // 128, **f32)
         self.recv_ids = torch.empty(Rmax, **i32)
-        self.load_l = torch.empty(self.E_local, **i32)
+        self.load_l = torch.zeros(self.E_local, **i32)
+        self.load_all = torch.zeros(E, **i32)
         self.offs_l = torch.empty(self.E_local + 1, **i32)
         self.tok_of_l = torch.empty(Rmax, **i32)
         self.row_of_l = torch.empty(Rmax, **i32)
@@ -135,6 +143,8 @@ class EPMoELayer:
         self._all_to_all(self.recv_s[:R], self.send_s, recv_splits, send_splits)
         self._all_to_all(self.recv_ids[:R], self.send_ids, recv_splits, send_splits)
         # the local experts on the received rows, results back in received order
+        if R == 0:
+            self.load_l.zero_()
         if R > 0:
             dl = a.dims(R, H, E_l, 1, 1, 1, I, 1.0)
             a.moe_permute(dl, self.recv_ids[:R], self.recv_q[:R], self.recv_s[:R], self.load_l, self.offs_l,
@@ -152,3 +162,18 @@ class EPMoELayer:
                                        a.MOE_EPI_BF16, self.ysh, None, st)
         a.moe_combine(dd, self.y_back, self.row_of_s, self.topk_w, self.ysh, self.out)
         return self.out
+
+    def bias_update(self, gamma: float, bias: Optional[torch.Tensor] = None, stream=None):
+        """b += gamma * sign(T_all*K/E - load) with every expert's load over all
+        ranks' T tokens of the last forward (T_all = world * T), applied to the
+        routing bias (default) or to `bias`.  Collective: every rank calls it."""
+        W = self.world
+        if W == 1:
+            self.load_all.copy_(self.load_l)
+        else:
+            parts = [torch.empty_like(self.load_l) for _ in range(W)]
+            dist.all_gather(parts, self.load_l, group=self.group)
+            # parts[r][j] is the load of global expert j * world + r
+            self.load_all.copy_(torch.stack(parts, dim=1).reshape(-1))
+        self.abi.moe_bias_update(self.E, self.T * W, self.K, gamma, self.load_all,
+                                 self.e_bias if bias is None else bias, stream)

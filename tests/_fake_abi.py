@@ -89,3 +89,7 @@ def moe_combine(d, yperm, row_of, topk_w, yshared, out, out_f32=None, stream=Non
     ysh = None if yshared is None else yshared.float().numpy()
     o = oracle.combine(yperm.float().numpy(), row_of.numpy(), w, ysh)
     out.copy_(torch.from_numpy(oracle.round_bf16(o)).to(out.dtype))
+
+
+def moe_bias_update(E, T, K, gamma, expert_load, e_bias, stream=None):
+    e_bias.copy_(torch.from_numpy(oracle.bias_update(e_bias.numpy(), expert_load.numpy(), T, K, gamma)))

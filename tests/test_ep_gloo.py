@@ -2,7 +2,8 @@
 (gloo), with the library calls replaced by their oracle-built CPU stand-ins
 (tests/_fake_abi.py): each rank holds the routed experts e with e % 2 == rank,
 routes its own tokens, and must produce exactly the oracle's single-process
-layer output for those tokens."""
+layer output for those tokens; the bias update from the all-gathered expert
+loads must equal the oracle's update from the loads of all ranks' tokens."""
 import os
 import socket
 
@@ -52,8 +53,20 @@ def _worker(rank, world, port, q):
         ref = oracle.moe_forward(x.float().numpy(), wr.numpy(), b.numpy(), oracle.LayerWeights(master), s.n_group,
                                  s.topk_group, K, s.rho)
         recv = int(layer.recv_counts.sum())
+        # bias update from the global loads: same on every rank, equal to the oracle's
+        gamma = 0.001
+        b0 = layer.e_bias.clone()
+        layer.bias_update(gamma)
+        s32 = oracle.router_scores(x_all.float().numpy(), wr.numpy(), None).astype(np.float32)
+        idx_all, _ = oracle.select_experts(s32, b0.numpy(), s.n_group, s.topk_group, K, s.rho)
+        load_all = np.bincount(idx_all.reshape(-1), minlength=E)
+        ref_b = oracle.bias_update(b0.numpy(), load_all, world * T, K, gamma)
+        same_b = bool(np.array_equal(layer.e_bias.numpy(), ref_b)) and bool(np.array_equal(
+            layer.load_all.numpy(), load_all))
+        moved = bool((layer.e_bias != b0).any())
         dist.destroy_process_group()
-        q.put((rank, bool(np.array_equal(out, ref["out"])), float(np.abs(out - ref["out"]).max()), recv))
+        q.put((rank, bool(np.array_equal(out, ref["out"])) and same_b and moved,
+               f"out {float(np.abs(out - ref['out']).max())} bias {same_b} moved {moved}", recv))
     except Exception as exc:                     # report instead of hanging the parent
         q.put((rank, False, repr(exc), -1))
 

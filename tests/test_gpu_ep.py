@@ -26,6 +26,13 @@ def test_ep_layer_one_rank_same_bits_as_layer(lib, shape):
     assert int(ep.status.item()) == 0
     assert torch.equal(got, ref)
     assert torch.equal(ep.topk_idx, layer.topk_idx)
+    # the bias update from the (here single-rank) global loads: same bits as the layer's
+    b_ep, b_layer = layer.e_bias.clone(), layer.e_bias.clone()
+    ep.bias_update(0.001, bias=b_ep)
+    layer.bias_update(0.001, bias=b_layer)
+    torch.cuda.synchronize()
+    assert torch.equal(ep.load_all, layer.load)
+    assert torch.equal(b_ep, b_layer)
 
 
 def test_ep_split_and_scatter(lib):
