@@ -196,6 +196,26 @@ class MoELayer:
                         self.out_f32 if out_f32 else None, stream)
         return out
 
+    def capture_graph(self, x: torch.Tensor, gamma: Optional[float] = None,
+                      bias: Optional[torch.Tensor] = None) -> "torch.cuda.CUDAGraph":
+        """Capture one forward on the device tensor x (and, with gamma, the bias
+        update into `bias` or the routing bias) as a CUDA graph.  Replaying it
+        reruns the same kernels on whatever x then holds, writing self.out,
+        without per-launch host work.  One eager forward on a side stream runs
+        first, so that every kernel's one-time setup happens outside the
+        capture."""
+        side = torch.cuda.Stream(device=x.device)
+        side.wait_stream(torch.cuda.current_stream(x.device))
+        with torch.cuda.stream(side):
+            self.forward(x)
+        torch.cuda.current_stream(x.device).wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.forward(x)
+            if gamma is not None:
+                self.bias_update(gamma, bias=bias)
+        return graph
+
     def refresh_router(self, stream=None):
         """Split the router weights into the pieces the forward routes with."""
         abi.moe_router_split(self.w_router, self.w_pieces, stream)

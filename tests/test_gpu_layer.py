@@ -210,3 +210,29 @@ def test_layer_gather_equals_materialised(lib, shape):
     for name in ("topk_idx", "load", "offsets", "tok_of", "row_of", "xq", "xs", "actq", "acts", "yperm"):
         assert torch.equal(getattr(lay_g, name), getattr(lay_m, name)), name
     assert torch.equal(og, om)
+
+
+def test_layer_cuda_graph_replay(lib):
+    """A captured forward + bias update replays the same kernels: same output
+    bits as the eager forward, on new input written into the captured buffer,
+    and the same bias update."""
+    shape = synth.MID
+    layer, master, wr, b = build_layer(lib, shape, device="cpu")
+    xs = [cuda(synth.activations(shape.T, shape.H, 100 + i, shape.x_outlier_frac)) for i in range(2)]
+    eager, bias_eager = [], []
+    for x in xs:
+        bb = layer.e_bias.clone()
+        eager.append(layer.forward(x).clone())
+        layer.bias_update(0.001, bias=bb)
+        bias_eager.append(bb)
+    x_static = xs[0].clone()
+    b_graph = layer.e_bias.clone()
+    graph = layer.capture_graph(x_static, gamma=0.001, bias=b_graph)
+    for i, x in enumerate(xs):
+        x_static.copy_(x)
+        b_graph.copy_(layer.e_bias)
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(layer.out, eager[i])
+        assert torch.equal(b_graph, bias_eager[i])
+    assert int(layer.status.item()) == 0
