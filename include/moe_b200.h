@@ -299,6 +299,37 @@ int moe_ep_split(const int32_t *topk_idx, int64_t n, int32_t E, int32_t world, i
                  int32_t *local_idx, int32_t *status, void *stream);
 int moe_ep_scatter(const int32_t *row_of, const int32_t *values, int64_t n, int32_t *out, void *stream);
 
+/* Node-limited dispatch: each token sent at most once to each rank
+ * ([report-walkthrough] section 3.4: a token reaches at most M nodes, picked by
+ * group; section 4.1: it crosses to a node once and is forwarded there to the
+ * experts it selected on that node; [infra-answer]: grouped routing caps the
+ * nodes per token at 4, halving cross-node traffic).  Placement:
+ *   MOE_EP_CYCLIC  expert e on rank e % world as local expert e / world
+ *   MOE_EP_BLOCK   expert e on rank e / (E/world) as local expert e % (E/world)
+ *                  (with world = n_group, rank = group: topk_group ranks at most)
+ * moe_ep_plan, for T tokens x K slots (K <= 32, E % world == 0):
+ *   dest_rank[t*K+k] = rank of slot k's expert if no earlier slot of token t has
+ *                      that rank, else -1 (not dispatched)
+ *   for a dispatched slot i = t*K+k, row i of meta_ids / meta_w [T*K, K]:
+ *     meta_ids[i, j] = local expert id of slot j if slot j's expert is on
+ *                      dest_rank[i], else -1;  meta_w[i, j] = topk_w[t, j] or 0
+ *   (rows of slots that are not dispatched hold -1 / 0).
+ * An expert index outside [0, E) raises MOE_FLAG_BAD_INDEX; that slot is not
+ * dispatched.  Dispatch is then moe_permute with dest_rank as its indices and
+ * the ranks as groups (status NULL: the -1 slots are skipped, not errors), the
+ * metadata moved into its order with moe_ep_scatter_rows; on the receiver the
+ * rows' meta_ids are the indices of a moe_permute over the local experts, and
+ * moe_combine with meta_w sums each row's experts.
+ * moe_ep_scatter_rows: out[row_of[i], :] = values[i, :] for rows of `width`
+ *                      int32 (fp32 bit patterns move unchanged) with row_of[i] >= 0. */
+#define MOE_EP_CYCLIC 0
+#define MOE_EP_BLOCK 1
+int moe_ep_plan(const int32_t *topk_idx, const float *topk_w, int64_t T, int32_t K, int32_t E, int32_t world,
+                int32_t placement, int32_t *dest_rank, int32_t *meta_ids, float *meta_w, int32_t *status,
+                void *stream);
+int moe_ep_scatter_rows(const int32_t *row_of, const int32_t *values, int64_t n, int32_t width, int32_t *out,
+                        void *stream);
+
 /* Sequence-wise balance loss and expert-load entropy ([report-walkthrough]
  * section 3.3: a complementary per-sequence balance loss with a very small
  * coefficient; aux_loss_alpha 0.001 in [repro-guide] section 3).  For each

@@ -37,7 +37,7 @@ from .fp8 import (E4M3_MAX, e4m3_encode, e4m3_decode, e4m3_encode_scalar, e4m3_d
                   round_bf16, quant_1x128, quant_128x128, dequant_1x128, dequant_128x128)
 from .routing import (router_scores, select_experts, select_experts_bruteforce,
                       expert_load, bias_update, seq_balance_loss, load_entropy)
-from .dispatch import permute, unpermute_rows, combine
+from .dispatch import permute, unpermute_rows, combine, combine_by_rank
 from .expert import (gemm_blockscaled, grouped_gemm_blockscaled, silu, swiglu,
                      swiglu_requant, expert_ffn)
 from .layer import LayerWeights, quantize_layer_weights, moe_forward, moe_forward_tokens
@@ -47,7 +47,7 @@ __all__ = [
     "round_bf16", "quant_1x128", "quant_128x128", "dequant_1x128", "dequant_128x128",
     "router_scores", "select_experts", "select_experts_bruteforce", "expert_load", "bias_update",
     "seq_balance_loss", "load_entropy",
-    "permute", "unpermute_rows", "combine",
+    "permute", "unpermute_rows", "combine", "combine_by_rank",
     "gemm_blockscaled", "grouped_gemm_blockscaled", "silu", "swiglu", "swiglu_requant", "expert_ffn",
     "LayerWeights", "quantize_layer_weights", "moe_forward", "moe_forward_tokens",
 ]

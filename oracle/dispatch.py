@@ -16,6 +16,8 @@ from __future__ import annotations
 
 import numpy as np
 
+from .fp8 import round_bf16
+
 
 def permute(idx, E: int):
     """Stable counting sort of the (token, slot) pairs by expert.
@@ -59,6 +61,35 @@ def combine(yperm, row_of, w, yshared=None):
     out = np.zeros((T, y.shape[1]), dtype=np.float64)
     for k in range(K):
         out += w64[:, k:k + 1] * y[r[:, k]]
+    if yshared is not None:
+        out += np.asarray(yshared, dtype=np.float64)
+    return out
+
+
+def combine_by_rank(yperm, row_of, w, rank, yshared=None):
+    """Node-limited combine: out[t] = sum over the ranks r that token t selected
+    of bf16( sum_{k : rank[t,k] = r} w[t,k] * yperm[row_of[t,k]] ) (+ yshared[t]),
+    float64 sums.
+
+    [report-walkthrough] section 3.4 sends a token at most once to each node it
+    selected; section 4.1 has the node compute the token's experts there and
+    accumulate their results while the combine forwards them back.  Each rank's
+    gated partial sum is the row that crosses back; it is stored in bf16, the
+    precision of the expert rows it sums (R12), and the source adds the partials.
+    rank int [T, K]: the rank of each slot's expert."""
+    w64 = np.asarray(w, dtype=np.float64)
+    T, K = w64.shape
+    y = np.asarray(yperm, dtype=np.float64)
+    r = np.asarray(row_of, dtype=np.int64).reshape(T, K)
+    rk = np.asarray(rank, dtype=np.int64).reshape(T, K)
+    out = np.zeros((T, y.shape[1]), dtype=np.float64)
+    for t in range(T):
+        for dest in sorted(set(int(v) for v in rk[t])):
+            part = np.zeros(y.shape[1], dtype=np.float64)
+            for k in range(K):
+                if rk[t, k] == dest:
+                    part += w64[t, k] * y[r[t, k]]
+            out[t] += round_bf16(part)
     if yshared is not None:
         out += np.asarray(yshared, dtype=np.float64)
     return out

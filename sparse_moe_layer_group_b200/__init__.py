@@ -10,7 +10,8 @@ from ._abi import (MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_REQUANT, MOE_FLAG_B
                    fp8_grouped_gemm_blockscaled, fp8_grouped_gemm_blockscaled_gather, fp8_quant_128x128, fp8_quant_1x128, moe_bias_update,
                    moe_balance_stats, moe_combine, moe_permute, moe_route, moe_route_pieces, moe_route_select,
                    moe_router_pieces_bytes, moe_router_split, swiglu_requant, fp8_quant_128x1_grouped,
-                   fp8_grouped_gemm_wgrad, wgrad_capacities, moe_ep_split, moe_ep_scatter,
+                   fp8_grouped_gemm_wgrad, wgrad_capacities, moe_ep_split, moe_ep_scatter, moe_ep_plan,
+                   moe_ep_scatter_rows, MOE_EP_CYCLIC, MOE_EP_BLOCK,
                    workspace_size)
 from .ep import EPMoELayer
 from .layer import LAUNCHES_PER_FORWARD, MoELayer, QuantWeights
@@ -20,7 +21,8 @@ __all__ = [
     "moe_route_select", "moe_route_pieces", "moe_router_split", "moe_router_pieces_bytes", "moe_permute", "fp8_grouped_gemm_blockscaled",
     "fp8_grouped_gemm_blockscaled_gather", "swiglu_requant", "moe_combine",
     "moe_bias_update", "moe_balance_stats", "fp8_quant_128x1_grouped", "fp8_grouped_gemm_wgrad",
-    "wgrad_capacities", "MoELayer", "QuantWeights", "LAUNCHES_PER_FORWARD",
+    "wgrad_capacities", "moe_ep_split", "moe_ep_scatter", "moe_ep_plan", "moe_ep_scatter_rows",
+    "MOE_EP_CYCLIC", "MOE_EP_BLOCK", "EPMoELayer", "MoELayer", "QuantWeights", "LAUNCHES_PER_FORWARD",
     "MOE_EPI_BF16", "MOE_EPI_F32", "MOE_EPI_SWIGLU_REQUANT",
     "MOE_FLAG_NONFINITE", "MOE_FLAG_BAD_INDEX", "MOE_FLAG_TIMEOUT", "MOE_FLAG_BAD_OFFSETS",
 ]

@@ -19,6 +19,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUD
 MOE_FLAG_NONFINITE, MOE_FLAG_BAD_INDEX, MOE_FLAG_TIMEOUT, MOE_FLAG_BAD_OFFSETS = 1, 2, 4, 8
 MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_REQUANT = 0, 1, 2
 MOE_GEMM_SINGLE_CTA, MOE_GEMM_PAIR_CTA = 0x100, 0x200
+MOE_EP_CYCLIC, MOE_EP_BLOCK = 0, 1
 
 
 class MoEError(RuntimeError):
@@ -72,6 +73,8 @@ _SIGS = {
     "moe_bias_update": (ctypes.c_int, [_I32, _I64, _I32, _F, _P, _P, _P]),
     "moe_ep_split": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P]),
     "moe_ep_scatter": (ctypes.c_int, [_P, _P, _I64, _P, _P]),
+    "moe_ep_plan": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P]),
+    "moe_ep_scatter_rows": (ctypes.c_int, [_P, _P, _I64, _I32, _P, _P]),
     "moe_balance_stats": (ctypes.c_int, [_DIMS, _P, _P, _P, _I32, ctypes.c_double, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -253,3 +256,18 @@ def moe_balance_stats(d, scores, topk_idx, expert_load, seq_len, alpha, seq_loss
     _check("moe_balance_stats", _lib.moe_balance_stats(ctypes.byref(d), _ptr(scores), _ptr(topk_idx),
                                                        _ptr(expert_load), int(seq_len), float(alpha),
                                                        _ptr(seq_loss), _ptr(entropy), _stream(stream)))
+
+
+def moe_ep_plan(topk_idx, topk_w, E, world, placement, dest_rank, meta_ids, meta_w, status=None, stream=None):
+    T, K = topk_idx.shape
+    _check("moe_ep_plan", _lib.moe_ep_plan(_ptr(topk_idx), _ptr(topk_w), int(T), int(K), int(E), int(world),
+                                           int(placement),
+                                           _ptr(dest_rank), _ptr(meta_ids), _ptr(meta_w), _ptr(status),
+                                           _stream(stream)))
+
+
+def moe_ep_scatter_rows(row_of, values, out, stream=None):
+    """out[row_of[i], :] = values[i, :] for int32 (or fp32, moved as bits) rows."""
+    n, width = values.shape
+    _check("moe_ep_scatter_rows", _lib.moe_ep_scatter_rows(_ptr(row_of), _ptr(values), int(n), int(width),
+                                                           _ptr(out), _stream(stream)))

@@ -1,6 +1,23 @@
 """Expert-parallel DeepSeekMoE layer forward: the routed experts spread over the
 ranks of a process group, each rank routing its own tokens.
 
+Two dispatch forms:
+
+* per slot (dedupe=False): every (token, slot) pair is sent to the rank of its
+  expert as its own row, computed there and returned as its own row; the
+  source combines them exactly as the single-GPU layer (same bits).
+* node-limited (dedupe=True, the default): a token crosses to each rank it
+  selected at most once (section 3.4 of the walkthrough: a token reaches at
+  most M nodes; section 4.1: it crosses once and is forwarded there to its
+  experts).  The row carries the local expert ids and gates of all of the
+  token's slots on that rank; the receiving rank computes them and sums them
+  (gated) into one partial row, which crosses back in bf16; the source adds the
+  partial rows and the shared expert.  With placement "block" (expert e on rank
+  e // (E/world)) and world == n_group, a rank is a routing group, so a token
+  crosses to at most topk_group ranks.  The extra bf16 rounding of each
+  partial makes this form equal to the oracle's combine_by_rank, not to the
+  single-GPU layer's bits.
+
 The "DeepSeek-V3 technical report" walkthrough (2kiu.com), section 4.1, runs
 the routed experts with expert parallelism: every device holds a subset of the
 experts, a token's rows are dispatched to the devices of its experts, processed
@@ -48,13 +65,20 @@ from .layer import QuantWeights
 class EPMoELayer:
     """One rank's part of an expert-parallel layer for T tokens per rank.
 
-    weights holds this rank's routed experts (local ids 0..E/world-1, i.e.
-    global experts rank, rank + world, ...) followed by the shared expert."""
+    weights holds this rank's routed experts in local order followed by the
+    shared expert: with placement "cyclic" the global experts rank, rank +
+    world, ...; with "block" the experts rank * E/world .. (rank + 1) * E/world - 1."""
 
     def __init__(self, T: int, H: int, E: int, K: int, n_group: int, topk_group: int, I: int, rho: float,
                  w_router: torch.Tensor, e_bias: torch.Tensor, weights: QuantWeights, group=None,
-                 router_offset: Optional[torch.Tensor] = None, device="cuda", abi=None):
+                 router_offset: Optional[torch.Tensor] = None, device="cuda", abi=None, dedupe: bool = True,
+                 placement: str = "block"):
         self.abi = _abi if abi is None else abi
+        if placement not in ("cyclic", "block"):
+            raise ValueError("placement is 'cyclic' or 'block'")
+        if not dedupe and placement != "cyclic":
+            raise ValueError("the per-slot dispatch places experts cyclically")
+        self.dedupe, self.placement = dedupe, placement
         self.group = group
         self.world = dist.get_world_size(group) if (group is not None or dist.is_initialized()) else 1
         self.rank = dist.get_rank(group) if self.world > 1 or dist.is_initialized() else 0
@@ -75,7 +99,8 @@ class EPMoELayer:
         self.w_pieces = torch.empty(self.abi.moe_router_pieces_bytes(E, H) // 2, **bf)
         self.abi.moe_router_split(w_router, self.w_pieces)
         ws_bytes = max(self.abi.workspace_size(self.d),
-                       self.abi.workspace_size(self.abi.dims(Rmax, H, self.E_local, 1, 1, 1, I, rho)), 256)
+                       self.abi.workspace_size(self.abi.dims(Rmax, H, self.E_local, 1, 1, 1, I, rho)),
+                       self.abi.workspace_size(self.abi.dims(W * T, H, self.E_local, K, 1, 1, I, rho)), 256)
         self.ws = torch.empty((ws_bytes + 255) // 256 * 256, **u8)
         self.topk_idx = torch.empty(T, K, **i32)
         self.topk_w = torch.empty(T, K, **f32)
@@ -107,6 +132,17 @@ class EPMoELayer:
         self.yperm_l = torch.empty(Rmax, H, **bf)
         self.y_recv = torch.empty(Rmax, H, **bf)
         self.ones = torch.ones(Rmax, **f32)
+        if dedupe:
+            # node-limited dispatch: at most one row per (token, rank) each way,
+            # with the K slots' local ids and gates riding along
+            self.meta_ids = torch.empty(TK, K, **i32)
+            self.meta_w = torch.empty(TK, K, **f32)
+            self.send_mids = torch.empty(TK, K, **i32)
+            self.send_mw = torch.empty(TK, K, **f32)
+            self.recv_mids = torch.empty(W * T, K, **i32)
+            self.recv_mw = torch.empty(W * T, K, **f32)
+            self.row_of_p = torch.empty(W * T * K, **i32)
+            self.ones_tk = torch.ones(T, K, **f32)
         self.y_back = torch.empty(TK, H, **bf)
         self.offs_sh = torch.tensor([0, T], **i32)
         self.actq_s = torch.empty(T, I, **u8)
@@ -124,6 +160,8 @@ class EPMoELayer:
         dist.all_to_all_single(out, inp, out_splits, in_splits, group=self.group)
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:
+        if self.dedupe:
+            return self._forward_node_limited(x)
         a, T, H, K, I, E_l = self.abi, self.T, self.H, self.K, self.I, self.E_local
         st, qw = self.status, self.qw
         a.moe_route_pieces(self.d, x, self.w_pieces, self.e_bias, self.router_offset, self.topk_idx, self.topk_w,
@@ -163,6 +201,53 @@ class EPMoELayer:
         a.moe_combine(dd, self.y_back, self.row_of_s, self.topk_w, self.ysh, self.out)
         return self.out
 
+    def _forward_node_limited(self, x: torch.Tensor) -> torch.Tensor:
+        a, T, H, K, I, E_l, W = self.abi, self.T, self.H, self.K, self.I, self.E_local, self.world
+        st, qw = self.status, self.qw
+        a.moe_route_pieces(self.d, x, self.w_pieces, self.e_bias, self.router_offset, self.topk_idx, self.topk_w,
+                           self.scores, self.ws, st)
+        a.fp8_quant_1x128(x, self.xq, self.xs, st)
+        # dispatch plan: one row per (token, rank), the first slot of each rank
+        # stands for it; rows grouped by destination rank
+        a.moe_ep_plan(self.topk_idx, self.topk_w, self.E, W,
+                      a.MOE_EP_BLOCK if self.placement == "block" else a.MOE_EP_CYCLIC,
+                      self.dest, self.meta_ids, self.meta_w, st)
+        dd = a.dims(T, H, W, K, 1, 1, I, 1.0)
+        # status None: the -1 entries of dest are slots that are not sent
+        a.moe_permute(dd, self.dest, self.xq, self.xs, self.send_load, self.send_offs, self.tok_of_s, self.row_of_s,
+                      self.send_q, self.send_s, self.ws, None)
+        a.moe_ep_scatter_rows(self.row_of_s, self.meta_ids, self.send_mids)
+        a.moe_ep_scatter_rows(self.row_of_s, self.meta_w.view(torch.int32), self.send_mw.view(torch.int32))
+        self._all_to_all(self.recv_counts, self.send_load, [1] * W, [1] * W)
+        send_splits = [int(v) for v in self.send_load.tolist()]
+        recv_splits = [int(v) for v in self.recv_counts.tolist()]
+        R = sum(recv_splits)
+        S = sum(send_splits)
+        self._all_to_all(self.recv_q[:R], self.send_q[:S], recv_splits, send_splits)
+        self._all_to_all(self.recv_s[:R], self.send_s[:S], recv_splits, send_splits)
+        self._all_to_all(self.recv_mids[:R], self.send_mids[:S], recv_splits, send_splits)
+        self._all_to_all(self.recv_mw[:R], self.send_mw[:S], recv_splits, send_splits)
+        # the local experts of every received row, then each row's gated sum
+        if R == 0:
+            self.load_l.zero_()
+        else:
+            dl = a.dims(R, H, E_l, K, 1, 1, I, 1.0)
+            a.moe_permute(dl, self.recv_mids[:R], self.recv_q[:R], self.recv_s[:R], self.load_l, self.offs_l,
+                          self.tok_of_l[:R * K], self.row_of_p[:R * K], self.aq_l, self.as_l, self.ws, None)
+            a.fp8_grouped_gemm_blockscaled(E_l, self.offs_l, R * K, 2 * I, H, self.aq_l, self.as_l, qw.w13, qw.s13,
+                                           a.MOE_EPI_SWIGLU_REQUANT, self.actq_l, self.acts_l, st)
+            a.fp8_grouped_gemm_blockscaled(E_l, self.offs_l, R * K, H, I, self.actq_l, self.acts_l, qw.w2, qw.s2,
+                                           a.MOE_EPI_BF16, self.yperm_l, None, st)
+            a.moe_combine(dl, self.yperm_l, self.row_of_p[:R * K], self.recv_mw[:R], None, self.y_recv[:R])
+        self._all_to_all(self.y_back[:S], self.y_recv[:R], send_splits, recv_splits)
+        # the shared expert on this rank's tokens, then the partial rows and the shared row
+        a.fp8_grouped_gemm_blockscaled(1, self.offs_sh, T, 2 * I, H, self.xq, self.xs, qw.w13[E_l:], qw.s13[E_l:],
+                                       a.MOE_EPI_SWIGLU_REQUANT, self.actq_s, self.acts_s, st)
+        a.fp8_grouped_gemm_blockscaled(1, self.offs_sh, T, H, I, self.actq_s, self.acts_s, qw.w2[E_l:], qw.s2[E_l:],
+                                       a.MOE_EPI_BF16, self.ysh, None, st)
+        a.moe_combine(dd, self.y_back, self.row_of_s, self.ones_tk, self.ysh, self.out)
+        return self.out
+
     def bias_update(self, gamma: float, bias: Optional[torch.Tensor] = None, stream=None):
         """b += gamma * sign(T_all*K/E - load) with every expert's load over all
         ranks' T tokens of the last forward (T_all = world * T), applied to the
@@ -173,7 +258,11 @@ class EPMoELayer:
         else:
             parts = [torch.empty_like(self.load_l) for _ in range(W)]
             dist.all_gather(parts, self.load_l, group=self.group)
-            # parts[r][j] is the load of global expert j * world + r
-            self.load_all.copy_(torch.stack(parts, dim=1).reshape(-1))
+            if self.placement == "block":
+                # parts[r][j] is the load of global expert r * E/world + j
+                self.load_all.copy_(torch.cat(parts))
+            else:
+                # parts[r][j] is the load of global expert j * world + r
+                self.load_all.copy_(torch.stack(parts, dim=1).reshape(-1))
         self.abi.moe_bias_update(self.E, self.T * W, self.K, gamma, self.load_all,
                                  self.e_bias if bias is None else bias, stream)

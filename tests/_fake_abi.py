@@ -9,7 +9,8 @@ import numpy as np
 import torch
 
 import oracle
-from sparse_moe_layer_group_b200._abi import MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_REQUANT, dims  # noqa: F401
+from sparse_moe_layer_group_b200._abi import (MOE_EP_BLOCK, MOE_EP_CYCLIC, MOE_EPI_BF16, MOE_EPI_F32,  # noqa: F401
+                                              MOE_EPI_SWIGLU_REQUANT, dims)
 
 _WR = {}
 
@@ -50,13 +51,31 @@ def moe_ep_split(topk_idx, E, world, dest_rank, local_idx, status=None, stream=N
     local_idx.copy_(torch.from_numpy((e // world).astype(np.int32)))
 
 
+def _permute_skipping(idx, E):
+    """oracle.permute over the entries in [0, E); the others get row_of = -1
+    (the library's treatment of an index it does not dispatch)."""
+    T, K = idx.shape
+    ok = (idx >= 0) & (idx < E)
+    if ok.all():
+        return oracle.permute(idx, E)
+    pairs = sorted((int(idx[t, k]), t, k) for t in range(T) for k in range(K) if ok[t, k])
+    load = np.bincount([e for e, _, _ in pairs], minlength=E).astype(np.int32)
+    offs = np.concatenate([[0], np.cumsum(load)]).astype(np.int32)
+    tok = np.zeros(T * K, dtype=np.int32)
+    row = np.full(T * K, -1, dtype=np.int32)
+    for r, (_, t, k) in enumerate(pairs):
+        tok[r] = t
+        row[t * K + k] = r
+    return load, offs, tok[:len(pairs)], row
+
+
 def moe_permute(d, topk_idx, xq, xs, expert_load, expert_offsets, tok_of, row_of, aq, as_, ws, status=None,
                 stream=None):
     idx = topk_idx.reshape(d.T, d.K).numpy()
-    load, offs, tok, row = oracle.permute(idx, d.E)
+    load, offs, tok, row = _permute_skipping(idx, d.E)
     expert_load.copy_(torch.from_numpy(load))
     expert_offsets.copy_(torch.from_numpy(offs))
-    tok_of.copy_(torch.from_numpy(tok))
+    tok_of[:len(tok)].copy_(torch.from_numpy(tok))
     row_of.copy_(torch.from_numpy(row))
     if aq is not None:
         t = torch.from_numpy(tok.astype(np.int64))
@@ -85,11 +104,44 @@ def fp8_grouped_gemm_blockscaled(G, group_offsets, m_capacity, N, K, A, sA, B, s
 
 
 def moe_combine(d, yperm, row_of, topk_w, yshared, out, out_f32=None, stream=None):
-    w = topk_w.reshape(d.T, d.K).numpy()
+    w = topk_w.reshape(d.T, d.K).numpy().copy()
+    r = row_of.numpy().astype(np.int64).copy()
+    skip = r < 0                                  # slots the library's combine skips
+    w.reshape(-1)[skip] = 0.0
+    r[skip] = 0
     ysh = None if yshared is None else yshared.float().numpy()
-    o = oracle.combine(yperm.float().numpy(), row_of.numpy(), w, ysh)
+    o = oracle.combine(yperm.float().numpy(), r, w, ysh)
     out.copy_(torch.from_numpy(oracle.round_bf16(o)).to(out.dtype))
 
 
 def moe_bias_update(E, T, K, gamma, expert_load, e_bias, stream=None):
     e_bias.copy_(torch.from_numpy(oracle.bias_update(e_bias.numpy(), expert_load.numpy(), T, K, gamma)))
+
+
+def moe_ep_plan(topk_idx, topk_w, E, world, placement, dest_rank, meta_ids, meta_w, status=None, stream=None):
+    idx = topk_idx.numpy().astype(np.int64)
+    T, K = idx.shape
+    El = E // world
+    rank = idx // El if placement == MOE_EP_BLOCK else idx % world
+    local = idx % El if placement == MOE_EP_BLOCK else idx // world
+    dest = np.full(T * K, -1, dtype=np.int32)
+    mid = np.full((T * K, K), -1, dtype=np.int32)
+    mw = np.zeros((T * K, K), dtype=np.float32)
+    w = topk_w.numpy()
+    for t in range(T):
+        for k in range(K):
+            if rank[t, k] in rank[t, :k]:
+                continue
+            dest[t * K + k] = rank[t, k]
+            on = rank[t] == rank[t, k]
+            mid[t * K + k, on] = local[t, on]
+            mw[t * K + k, on] = w[t, on]
+    dest_rank.copy_(torch.from_numpy(dest))
+    meta_ids.copy_(torch.from_numpy(mid))
+    meta_w.copy_(torch.from_numpy(mw))
+
+
+def moe_ep_scatter_rows(row_of, values, out, stream=None):
+    r = row_of.numpy().astype(np.int64)
+    ok = r >= 0
+    out[torch.from_numpy(r[ok])] = values[torch.from_numpy(ok)]

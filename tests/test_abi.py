@@ -108,3 +108,22 @@ def test_wgrad_host_validation():
     # NULL operands
     assert L.fp8_grouped_gemm_wgrad(2, 16, 4, 128, 128, None, 16, 16, 16, 128, 2, 16, None, None) == \
         a.MOE_ERR_INVALID_ARG
+
+
+def test_python_bindings_marshal_zero_size_calls():
+    """The Python binding of each expert-parallel call passes the argument count
+    and types the C entry point declares (zero-size calls return before any
+    device work, so this runs without a GPU)."""
+    import torch
+    from sparse_moe_layer_group_b200 import _abi as a
+    i32, f32 = torch.int32, torch.float32
+    idx, w = torch.empty(0, 8, dtype=i32), torch.empty(0, 8, dtype=f32)
+    a.moe_ep_plan(idx, w, 16, 2, a.MOE_EP_BLOCK, torch.empty(0, dtype=i32), torch.empty(0, 8, dtype=i32),
+                  torch.empty(0, 8, dtype=f32), None, 0)
+    a.moe_ep_scatter_rows(torch.empty(0, dtype=i32), torch.empty(0, 4, dtype=i32), torch.empty(0, 4, dtype=i32), 0)
+    a.moe_ep_split(torch.empty(0, 8, dtype=i32), 16, 2, torch.empty(0, dtype=i32), torch.empty(0, dtype=i32), None, 0)
+    a.moe_ep_scatter(torch.empty(0, dtype=i32), torch.empty(0, dtype=i32), torch.empty(0, dtype=i32), 0)
+    with pytest.raises(a.MoEError):
+        a.moe_ep_plan(torch.empty(2, 8, dtype=i32), torch.empty(2, 8, dtype=f32), 16, 3, a.MOE_EP_BLOCK,
+                      torch.empty(16, dtype=i32), torch.empty(16, 8, dtype=i32), torch.empty(16, 8, dtype=f32),
+                      None, 0)                            # 16 experts do not divide over 3 ranks

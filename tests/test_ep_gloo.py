@@ -17,7 +17,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, q):
+def _worker(rank, world, port, q, dedupe=False):
     try:
         os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
         import datetime
@@ -38,8 +38,10 @@ def _worker(rank, world, port, q):
             rows, cols = (2 * I, H) if kind == "w13" else (H, I)
             return synth.expert_weight(rows, cols, s.w_std, synth.seed_of(s, tid, max(e, 0))).float().numpy()
 
-        # this rank's routed experts (global e = l * world + rank) and the shared one, quantised by the oracle
-        mine = [l * world + rank for l in range(E // world)] + [-1]
+        # this rank's routed experts and the shared one, quantised by the oracle: per-slot
+        # dispatch places expert e on rank e % world, node-limited dispatch on rank e // (E/world)
+        El = E // world
+        mine = ([rank * El + l for l in range(El)] if dedupe else [l * world + rank for l in range(El)]) + [-1]
         q13 = [oracle.quant_128x128(master("w13", e)) for e in mine]
         q2 = [oracle.quant_128x128(master("w2", e)) for e in mine]
         qw = QuantWeights(torch.from_numpy(np.stack([a for a, _ in q13])), torch.from_numpy(np.stack([b for _, b in q13])),
@@ -48,10 +50,18 @@ def _worker(rank, world, port, q):
         b = synth.expert_bias(E, s.bias_range, synth.seed_of(s, synth.BIAS))
         x_all = synth.activations(world * T, H, synth.seed_of(s, synth.X))
         x = x_all[rank * T:(rank + 1) * T].contiguous()
-        layer = EPMoELayer(T, H, E, K, s.n_group, s.topk_group, I, s.rho, wr, b, qw, device="cpu", abi=_fake_abi)
+        layer = EPMoELayer(T, H, E, K, s.n_group, s.topk_group, I, s.rho, wr, b, qw, device="cpu", abi=_fake_abi,
+                           dedupe=dedupe, placement="block" if dedupe else "cyclic")
         out = layer.forward(x).float().numpy()
         ref = oracle.moe_forward(x.float().numpy(), wr.numpy(), b.numpy(), oracle.LayerWeights(master), s.n_group,
                                  s.topk_group, K, s.rho)
+        if dedupe:
+            # each rank's gated partial sum crosses back in bf16
+            ref["out"] = oracle.round_bf16(oracle.combine_by_rank(ref["yperm"], ref["row_of"], ref["w"],
+                                                                  ref["idx"] // El, ref["ysh"]))
+            # a token crosses to each rank at most once
+            sent = int(layer.send_load.sum())
+            assert sent == sum(len(set(int(e) // El for e in row)) for row in ref["idx"])
         recv = int(layer.recv_counts.sum())
         # bias update from the global loads: same on every rank, equal to the oracle's
         gamma = 0.001
@@ -71,11 +81,19 @@ def _worker(rank, world, port, q):
         q.put((rank, False, repr(exc), -1))
 
 
-def test_expert_parallel_layer_matches_the_oracle_on_two_ranks():
+import pytest
+
+
+@pytest.mark.parametrize("dedupe,world", [(False, 2), (True, 2), (True, 4)])
+def test_expert_parallel_layer_matches_the_oracle_on_cpu_ranks(dedupe, world):
+    """Per-slot dispatch: the oracle's layer bit for bit.  Node-limited dispatch
+    (one row per token and rank, block placement): the oracle's layer with the
+    per-rank partial sums of combine_by_rank, bit for bit, and exactly one row
+    sent per (token, rank) pair."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, dedupe)) for r in range(world)]
     for p in procs:
         p.start()
     res = [q.get(timeout=300) for _ in procs]

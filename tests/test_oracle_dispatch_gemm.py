@@ -166,3 +166,34 @@ def test_layer_tokens_equal_full_layer():
     part = oracle.moe_forward_tokens(x[[1, 7, 11]], wr, bias, W, 2, 1, K, 2.5)
     assert np.array_equal(part["idx"], full["idx"][[1, 7, 11]])
     assert np.array_equal(part["out"], full["out"][[1, 7, 11]])
+
+
+# ---------------------------------------------------------------- node-limited combine
+def test_combine_by_rank_hand_example():
+    """Three slots, two ranks.  Rank 0's partial 1 + 2^-8 lies exactly halfway
+    between the bf16 neighbours 1 and 1 + 2^-7 and rounds to even (1.0); rank 1's
+    partial 2^-8 is exact; the source's float64 sum is 1 + 2^-8.  The single
+    combine of the same slots gives 1 + 2^-7."""
+    y = np.array([[1.0], [2.0 ** -8], [2.0 ** -8]])
+    row_of = np.array([0, 1, 2])
+    w = np.ones((1, 3), dtype=np.float32)
+    got = oracle.combine_by_rank(y, row_of, w, np.array([[0, 0, 1]]))
+    assert got[0, 0] == 1.0 + 2.0 ** -8
+    assert oracle.combine(y, row_of, w)[0, 0] == 1.0 + 2.0 ** -7
+
+
+def test_combine_by_rank_reduces_to_the_combine():
+    rng = np.random.default_rng(5)
+    T, K, H = 6, 4, 16
+    # bf16 rows and power-of-two gates: every product and every partial is exact in bf16
+    y = rng.integers(-8, 8, (T * K, H)).astype(np.float64)
+    w = (2.0 ** rng.integers(-3, 1, (T, K))).astype(np.float32)
+    row_of = rng.permutation(T * K)
+    ysh = oracle.round_bf16(rng.standard_normal((T, H)))
+    distinct = np.tile(np.arange(K), (T, 1))
+    assert np.array_equal(oracle.combine_by_rank(y, row_of, w, distinct, ysh), oracle.combine(y, row_of, w, ysh))
+    # one rank for every slot: the partial is the whole gated sum, rounded once
+    y2 = rng.standard_normal((T * K, H))
+    same = np.zeros((T, K), dtype=np.int64)
+    want = oracle.round_bf16(oracle.combine(y2, row_of, w)) + ysh
+    assert np.array_equal(oracle.combine_by_rank(y2, row_of, w, same, ysh), want)
