@@ -328,14 +328,18 @@ def run_gpu(args, rank, world, local):
 
     e2e_steps(max(1, args.warmup))
     torch.cuda.synchronize()
+    # a short idle first: right after the device-only region the GPU runs at
+    # power-capped clocks, which would be charged to the host copies
+    time.sleep(1.0)
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    h2d.wait_event(e0)
-    d2h.wait_event(e0)
-    e2e_steps(args.steps)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    with ClockSampler(local) as clk_e2e:
+        e0.record(stream)
+        h2d.wait_event(e0)
+        d2h.wait_event(e0)
+        e2e_steps(args.steps)
+        e1.record(stream)
+        torch.cuda.synchronize()
     e2e_ms = reduce_max(e0.elapsed_time(e1), world)
 
     if rank != 0:
@@ -377,7 +381,8 @@ def run_gpu(args, rank, world, local):
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * shape.H * 2, "d2h_bytes_per_step": T * shape.H * 2,
                 "how": "MoELayer.forward per step; pinned-host input copied in and output copied back on two "
-                       "copy streams overlapping the adjacent steps' compute (double-buffered device input/output)"},
+                       "copy streams overlapping the adjacent steps' compute (double-buffered device input/output)",
+                "clocks": clk_e2e.summary()},
         "w2_launch_ms": round(g2_ms, 4),
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
@@ -747,8 +752,10 @@ def run_case(args):
     """One kernel alone on a profiling-sized case (a few GB on the device):
     gemm1 = routed W13 GEMM with the SwiGLU+requant epilogue and gemm2 = routed
     W2 GEMM, both on 64 experts x 128 rows at the DSV3 hidden/intermediate
-    sizes (1.9 GB / 0.9 GB of weights, larger than L2); router = moe_route at
-    T=4096, H=7168, E=256."""
+    sizes (1.9 GB / 0.9 GB of weights, larger than L2); gemm1_gather = gemm1_skew
+    with its A rows gathered through a seeded row map from T/8 source rows (the
+    layer's fan-out of 8 slots per token); wgrad = the wgrad GEMM of W13 for 8
+    experts of ~144 rows (dW 0.94 GB); router = moe_route at T=4096, H=7168, E=256."""
     import sparse_moe_layer_group_b200 as moe
     abi = moe.abi
     shape = synth.DSV3
@@ -756,7 +763,7 @@ def run_case(args):
     E, rows = 64, 128
     dev = "cuda"
     ev = []
-    if args.case in ("gemm1", "gemm2", "gemm1_x256", "gemm1_skew"):
+    if args.case in ("gemm1", "gemm2", "gemm1_x256", "gemm1_skew", "gemm1_gather"):
         N, K = (H, I) if args.case == "gemm2" else (2 * I, H)
         w = torch.empty(E, N, K, dtype=torch.uint8, device=dev)
         sw = torch.empty(E, N // 128, K // 128, dtype=torch.float32, device=dev)
@@ -765,7 +772,7 @@ def run_case(args):
             abi.fp8_quant_128x128(m, w[e], sw[e])
         if args.case == "gemm1_x256":
             sizes = [2 * rows] * E
-        elif args.case == "gemm1_skew":
+        elif args.case in ("gemm1_skew", "gemm1_gather"):
             # log-normal expert loads with mean 128 rows (spread like an unbalanced router)
             g = synth.gen(11, "cpu")
             wts = torch.exp(0.6 * torch.randn(E, generator=g, dtype=torch.float64))
@@ -779,7 +786,15 @@ def run_case(args):
         abi.fp8_quant_1x128(a_bf, a, sa)
         offs = torch.tensor([0] + list(np.cumsum(sizes)), dtype=torch.int32, device=dev)
         mode = {"auto": 0, "single": abi.MOE_GEMM_SINGLE_CTA, "pair": abi.MOE_GEMM_PAIR_CTA}[args.gemm_mode]
-        if args.case != "gemm2":
+        if args.case == "gemm1_gather":
+            n_src = max(1, Mrows // 8)
+            a_map = torch.randint(0, n_src, (Mrows,), generator=synth.gen(13, "cpu"), dtype=torch.int32).to(dev)
+            src_q, src_s = a[:n_src].contiguous(), sa[:n_src].contiguous()
+            out = torch.empty(Mrows, N // 2, dtype=torch.uint8, device=dev)
+            so = torch.empty(Mrows, N // 256, dtype=torch.float32, device=dev)
+            run = lambda: abi.fp8_grouped_gemm_blockscaled_gather(E, offs, Mrows, N, K, src_q, src_s, a_map, w, sw,
+                                                                 abi.MOE_EPI_SWIGLU_REQUANT, out, so)
+        elif args.case != "gemm2":
             out = torch.empty(Mrows, N // 2, dtype=torch.uint8, device=dev)
             so = torch.empty(Mrows, N // 256, dtype=torch.float32, device=dev)
             run = lambda: abi.fp8_grouped_gemm_blockscaled(E, offs, Mrows, N, K, a, sa, w, sw,
@@ -790,6 +805,25 @@ def run_case(args):
                                                           abi.MOE_EPI_BF16 | mode, out)
         nbytes = E * N * K + Mrows * K + Mrows * (2 * N if args.case == "gemm2" else N // 2)
         flops = 2 * Mrows * N * K
+    elif args.case == "wgrad":
+        G, N, K = 8, 2 * I, H
+        g = synth.gen(14, "cpu")
+        sizes = (torch.full((G,), 144) + torch.randint(-40, 41, (G,), generator=g)).tolist()
+        M = int(sum(sizes))
+        offs = torch.tensor([0] + list(np.cumsum(sizes)), dtype=torch.int32, device=dev)
+        dy = synth.normal((M, N), 1.0, 81, device=dev, dtype=torch.bfloat16)
+        xx = synth.activations(M, K, 82, device=dev)
+        p_cap, t_cap = abi.wgrad_capacities(M, G)
+        dq = torch.empty(N, p_cap, dtype=torch.uint8, device=dev)
+        ds = torch.empty(t_cap, N, dtype=torch.float32, device=dev)
+        xq = torch.empty(K, p_cap, dtype=torch.uint8, device=dev)
+        xs = torch.empty(t_cap, K, dtype=torch.float32, device=dev)
+        dW = torch.empty(G, N, K, dtype=torch.float32, device=dev)
+        abi.fp8_quant_128x1_grouped(dy, offs, dq, ds)
+        abi.fp8_quant_128x1_grouped(xx, offs, xq, xs)
+        run = lambda: abi.fp8_grouped_gemm_wgrad(offs, M, dq, ds, xq, xs, dW)
+        nbytes = G * N * K * 4 + (N + K) * (p_cap + 4 * t_cap)
+        flops = 2 * M * N * K
     elif args.case == "router":
         T, E2 = shape.T, shape.E
         x = synth.activations(T, H, 1, device=dev)
@@ -830,7 +864,7 @@ def main():
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the prefill / decode / dense-GEMM legs reported under 'workloads'")
     ap.add_argument("--case", default=None,
-                    help="time one kernel alone: gemm1 | gemm1_x256 | gemm1_skew | gemm2 | router")
+                    help="time one kernel alone: gemm1 | gemm1_x256 | gemm1_skew | gemm1_gather | gemm2 | wgrad | router")
     ap.add_argument("--gemm-mode", default="auto", choices=["auto", "single", "pair"])
     args = ap.parse_args()
     if args.case:
