@@ -330,6 +330,62 @@ int moe_ep_plan(const int32_t *topk_idx, const float *topk_w, int64_t T, int32_t
 int moe_ep_scatter_rows(const int32_t *row_of, const int32_t *values, int64_t n, int32_t width, int32_t *out,
                         void *stream);
 
+/* The whole layer forward in one call ([report-walkthrough] sections 3.2 and
+ * 4.1: route -> dispatch -> expert MLP -> combine; section 4.3: FP8 steps):
+ * moe_route_pieces, fp8_quant_1x128, moe_permute, the two grouped GEMMs (the
+ * shared expert as group E) and moe_combine, then optionally moe_bias_update.
+ * Every buffer is the caller's (device memory, the sizes of the single calls):
+ *   w13, s13, w2, s2     the E+1 experts' E4M3 weights and scales (shared last)
+ *   w_pieces             moe_router_split's pieces of W_r; e_bias [E];
+ *                        router_offset [E] or NULL
+ *   topk_idx, topk_w [T,K], scores [T,E]
+ *   aq [T*K+T, H], as [T*K+T, H/128]  A of the first GEMM; its last T rows
+ *                        receive the quantised tokens
+ *   load [E]; offsets [E+2] with offsets[E+1] = T*K+T set by the caller once
+ *                        (moe_permute writes entries 0..E)
+ *   tok_of, row_of [T*K]; actq [T*K+T, I], acts [T*K+T, I/128]
+ *   yperm bf16 [T*K+T, H] (its last T rows: the shared expert's output)
+ *   ws, ws_bytes >= moe_workspace_size(dims); status (may be NULL)
+ *   bias_out [E] or NULL: when set, bias_out += gamma * sign(T*K/E - load)
+ *                        after the forward (the routing bias, or a copy of it)
+ * moe_layer_forward: x bf16 [T,H] -> out bf16 [T,H] (device), on `stream`.
+ * moe_layer_run_host: n batches from host memory: batch i's x_host[i] (pinned
+ * bf16 [T,H]) is uploaded on a stream of its own into x_dev[i % 2], the forward
+ * runs on `stream` into out_dev[i % 2], and out_host[i] (pinned) is downloaded
+ * on a third stream, so the copies of batches i+1 and i-1 overlap batch i's
+ * forward.  One cudaMemcpyAsync per copy.  Returns once everything is enqueued;
+ * `stream` completes after the last download.                                 */
+typedef struct {
+    moe_dims dims;
+    const uint8_t *w13;
+    const float *s13;
+    const uint8_t *w2;
+    const float *s2;
+    const void *w_pieces;
+    const float *e_bias;
+    const float *router_offset;
+    int32_t *topk_idx;
+    float *topk_w;
+    float *scores;
+    uint8_t *aq;
+    float *as;
+    int32_t *load;
+    int32_t *offsets;
+    int32_t *tok_of;
+    int32_t *row_of;
+    uint8_t *actq;
+    float *acts;
+    void *yperm;
+    void *ws;
+    size_t ws_bytes;
+    int32_t *status;
+    float *bias_out;
+    float gamma;
+} moe_layer;
+int moe_layer_forward(const moe_layer *layer, const void *x, void *out, void *stream);
+int moe_layer_run_host(const moe_layer *layer, const void *const *x_host, void *const *out_host, int32_t n,
+                       void *const *x_dev, void *const *out_dev, void *stream);
+
 /* Sequence-wise balance loss and expert-load entropy ([report-walkthrough]
  * section 3.3: a complementary per-sequence balance loss with a very small
  * coefficient; aux_loss_alpha 0.001 in [repro-guide] section 3).  For each

@@ -34,6 +34,17 @@ class MoeDims(ctypes.Structure):
                 ("I", ctypes.c_int32), ("routed_scaling_factor", ctypes.c_float)]
 
 
+_LAYER_PTRS = ("w13", "s13", "w2", "s2", "w_pieces", "e_bias", "router_offset", "topk_idx", "topk_w", "scores",
+               "aq", "as", "load", "offsets", "tok_of", "row_of", "actq", "acts", "yperm", "ws")
+
+
+class MoeLayerC(ctypes.Structure):
+    """moe_layer of the header: the dims and every device buffer of one layer."""
+    _fields_ = ([("dims", MoeDims)] + [(n, ctypes.c_void_p) for n in _LAYER_PTRS] +
+                [("ws_bytes", ctypes.c_size_t), ("status", ctypes.c_void_p), ("bias_out", ctypes.c_void_p),
+                 ("gamma", ctypes.c_float)])
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
@@ -76,6 +87,8 @@ _SIGS = {
     "moe_ep_plan": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P]),
     "moe_ep_scatter_rows": (ctypes.c_int, [_P, _P, _I64, _I32, _P, _P]),
     "moe_balance_stats": (ctypes.c_int, [_DIMS, _P, _P, _P, _I32, ctypes.c_double, _P, _P, _P]),
+    "moe_layer_forward": (ctypes.c_int, [ctypes.POINTER(MoeLayerC), _P, _P, _P]),
+    "moe_layer_run_host": (ctypes.c_int, [ctypes.POINTER(MoeLayerC), _P, _P, _I32, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -271,3 +284,34 @@ def moe_ep_scatter_rows(row_of, values, out, stream=None):
     n, width = values.shape
     _check("moe_ep_scatter_rows", _lib.moe_ep_scatter_rows(_ptr(row_of), _ptr(values), int(n), int(width),
                                                            _ptr(out), _stream(stream)))
+
+
+def moe_layer(d, buffers: dict, ws, status=None, bias_out=None, gamma: float = 0.0) -> MoeLayerC:
+    """Fill a moe_layer from device tensors: buffers maps each pointer field of
+    the header's struct (w13, s13, ..., yperm) to a tensor (router_offset may be None)."""
+    L = MoeLayerC()
+    L.dims = d
+    for n in _LAYER_PTRS:
+        setattr(L, n, _ptr(ws if n == "ws" else buffers.get(n)))
+    L.ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    L.status = _ptr(status)
+    L.bias_out = _ptr(bias_out)
+    L.gamma = float(gamma)
+    return L
+
+
+def moe_layer_forward(L: MoeLayerC, x, out, stream=None):
+    _check("moe_layer_forward", _lib.moe_layer_forward(ctypes.byref(L), _ptr(x), _ptr(out), _stream(stream)))
+
+
+def moe_layer_run_host(L: MoeLayerC, x_host, out_host, x_dev, out_dev, stream=None):
+    """Batches x_host[i] -> out_host[i] (pinned host tensors) through the device
+    double buffers x_dev[0..1], out_dev[0..1]; returns once enqueued."""
+    n = len(x_host)
+    if len(out_host) != n or len(x_dev) != 2 or len(out_dev) != 2:
+        raise ValueError("n host inputs and outputs, two device inputs and outputs")
+    xs = (ctypes.c_void_p * n)(*[_ptr(t) for t in x_host])
+    os_ = (ctypes.c_void_p * n)(*[_ptr(t) for t in out_host])
+    xd = (ctypes.c_void_p * 2)(*[_ptr(t) for t in x_dev])
+    od = (ctypes.c_void_p * 2)(*[_ptr(t) for t in out_dev])
+    _check("moe_layer_run_host", _lib.moe_layer_run_host(ctypes.byref(L), xs, os_, n, xd, od, _stream(stream)))

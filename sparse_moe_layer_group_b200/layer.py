@@ -196,6 +196,34 @@ class MoELayer:
                         self.out_f32 if out_f32 else None, stream)
         return out
 
+    def native(self, bias_out: Optional[torch.Tensor] = None, gamma: float = 0.0) -> "abi.MoeLayerC":
+        """The header's moe_layer for this layer's buffers (the materialised
+        path), for moe_layer_forward / moe_layer_run_host: the whole forward,
+        and the bias update into bias_out if given, behind one C call."""
+        if self.gather:
+            raise ValueError("the one-call forward runs the materialised path (gather=False)")
+        qw = self.qw
+        bufs = dict(w13=qw.w13, s13=qw.s13, w2=qw.w2, s2=qw.s2, w_pieces=self.w_pieces, e_bias=self.e_bias,
+                    router_offset=self.router_offset, topk_idx=self.topk_idx, topk_w=self.topk_w,
+                    scores=self.scores, aq=self.aq, load=self.load, offsets=self.offsets_all,
+                    tok_of=self.tok_of, row_of=self.row_of, actq=self.actq, acts=self.acts, yperm=self.yperm)
+        bufs["as"] = self.as_
+        return abi.moe_layer(self.d, bufs, self.ws, self.status, bias_out, gamma)
+
+    def forward_native(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None,
+                       bias_out: Optional[torch.Tensor] = None, gamma: float = 0.0) -> torch.Tensor:
+        """forward() as one C call (moe_layer_forward); same kernels, same bits."""
+        out = self.out if out is None else out
+        abi.moe_layer_forward(self.native(bias_out, gamma), x, out, stream)
+        return out
+
+    def run_host(self, x_host, out_host, x_dev, out_dev, stream=None, bias_out: Optional[torch.Tensor] = None,
+                 gamma: float = 0.0):
+        """Batches from pinned host memory through moe_layer_run_host: uploads and
+        downloads of neighbouring batches overlap each forward (two device input
+        and output buffers).  Returns once enqueued on `stream`."""
+        abi.moe_layer_run_host(self.native(bias_out, gamma), x_host, out_host, x_dev, out_dev, stream)
+
     def capture_graph(self, x: torch.Tensor, gamma: Optional[float] = None,
                       bias: Optional[torch.Tensor] = None) -> "torch.cuda.CUDAGraph":
         """Capture one forward on the device tensor x (and, with gamma, the bias

@@ -127,3 +127,24 @@ def test_python_bindings_marshal_zero_size_calls():
         a.moe_ep_plan(torch.empty(2, 8, dtype=i32), torch.empty(2, 8, dtype=f32), 16, 3, a.MOE_EP_BLOCK,
                       torch.empty(16, dtype=i32), torch.empty(16, 8, dtype=i32), torch.empty(16, 8, dtype=f32),
                       None, 0)                            # 16 experts do not divide over 3 ranks
+
+
+def test_layer_struct_layout_matches_the_header(tmp_path):
+    """The ctypes mirror of moe_layer has the header's size and field offsets
+    (a C program built from the header prints them)."""
+    import shutil
+    import subprocess
+    from sparse_moe_layer_group_b200 import _abi as a
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    fields = [f for f, _ in a.MoeLayerC._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "moe_b200.h"\nint main(void) {\n'
+                   '  printf("%zu\\n", sizeof(moe_layer));\n' +
+                   "".join(f'  printf("%zu\\n", offsetof(moe_layer, {f}));\n' for f in fields) + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()]
+    want = [ctypes.sizeof(a.MoeLayerC)] + [getattr(a.MoeLayerC, f).offset for f in fields]
+    assert got == want

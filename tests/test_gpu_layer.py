@@ -236,3 +236,36 @@ def test_layer_cuda_graph_replay(lib):
         assert torch.equal(layer.out, eager[i])
         assert torch.equal(b_graph, bias_eager[i])
     assert int(layer.status.item()) == 0
+
+
+@pytest.mark.parametrize("shape", [synth.MID, pytest.param(synth.DSV3, marks=pytest.mark.slow)])
+def test_layer_one_call_forward_and_host_runner(lib, shape):
+    """moe_layer_forward (the whole forward and the bias update behind one C
+    call) gives the Python-chained forward's bits; moe_layer_run_host on three
+    host batches gives each batch's forward output in its host buffer."""
+    dev = "cuda" if shape is synth.DSV3 else "cpu"
+    layer, master, wr, b = build_layer(lib, shape, device=dev)
+    xs = [synth.activations(shape.T, shape.H, 200 + i, shape.x_outlier_frac, device=dev) for i in range(3)]
+    ref, ref_b = [], []
+    for x in xs:
+        bb = layer.e_bias.clone()
+        ref.append(layer.forward(cuda(x)).clone())
+        layer.bias_update(0.001, bias=bb)
+        ref_b.append(bb)
+    torch.cuda.synchronize()
+    # one call on the device
+    b1 = layer.e_bias.clone()
+    out1 = torch.empty_like(ref[0])
+    layer.forward_native(cuda(xs[0]), out=out1, bias_out=b1, gamma=0.001)
+    torch.cuda.synchronize()
+    assert int(layer.status.item()) == 0
+    assert torch.equal(out1, ref[0]) and torch.equal(b1, ref_b[0])
+    # host batches: uploads, forwards and downloads overlapped, every output in place
+    x_host = [x.cpu().pin_memory() for x in xs]
+    out_host = [torch.full((shape.T, shape.H), float("nan"), dtype=torch.bfloat16).pin_memory() for _ in xs]
+    x_dev = [torch.empty_like(ref[0]) for _ in range(2)]
+    out_dev = [torch.empty_like(ref[0]) for _ in range(2)]
+    layer.run_host(x_host, out_host, x_dev, out_dev)
+    torch.cuda.synchronize()
+    for i in range(3):
+        assert torch.equal(out_host[i], ref[i].cpu()), f"batch {i}"
