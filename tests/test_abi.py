@@ -84,6 +84,12 @@ def test_host_validation_rejects_before_launch():
     assert gg(1, 16, 64, 256, 128, 16, 16, 0, 16, 16, 16, 0, 16, None, None, None) == a.MOE_ERR_INVALID_ARG
     assert gg(1, 16, 64, 256, 100, 16, 16, 8, 16, 16, 16, 0, 16, None, None, None) == a.MOE_ERR_INVALID_ARG
     assert gg(0, 16, 64, 256, 128, 16, 16, 8, 16, 16, 16, 0, 16, None, None, None) == 0
+    # one-call forward and host runner: the struct and buffers are required, n >= 0
+    assert L.moe_layer_forward(None, 16, 16, None) == a.MOE_ERR_INVALID_ARG
+    lay = a.MoeLayerC()
+    assert L.moe_layer_forward(ctypes.byref(lay), None, 16, None) == a.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_run_host(ctypes.byref(lay), None, None, -1, None, None, None) == a.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_run_host(ctypes.byref(lay), None, None, 0, None, None, None) == 0
     # zero-size work is a no-op
     assert L.fp8_grouped_gemm_blockscaled(0, 16, 64, 256, 128, 16, 16, 16, 16, 0, 16, None, None, None) == 0
     assert L.fp8_quant_1x128(16, 0, 128, 16, 16, None, None) == 0
