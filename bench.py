@@ -601,6 +601,49 @@ def leg_gather(layer, pk, iters: int = 10) -> dict:
     return out
 
 
+def leg_combine(layer, pk, iters: int = 10) -> dict:
+    """The second half of the DSV3 step two ways on the step's own routing and
+    activations: W2 storing its bf16 rows + the combine kernel (the layer's
+    default), and W2 with the combine in its epilogue (gates scattered into row
+    order, gated rows added into an fp32 accumulator at the L2) + the finishing
+    pass that rounds to bf16 and re-zeroes the accumulator (f3 combine half)."""
+    import sparse_moe_layer_group_b200 as moe
+    abi = moe.abi
+    T, H, K, I, E = layer.T, layer.H, layer.K, layer.I, layer.E
+    M = T * K + T
+    qw = layer.qw
+    row_gate = torch.ones(M, dtype=torch.float32, device="cuda")
+    acc = torch.zeros(T, H, dtype=torch.float32, device="cuda")
+    out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def stored():
+        abi.fp8_grouped_gemm_blockscaled(E + 1, layer.offsets_all, M, H, I, layer.actq, layer.acts, qw.w2, qw.s2,
+                                         abi.MOE_EPI_BF16, layer.yperm, None, st)
+        abi.moe_combine(layer.d, layer.yperm, layer.row_of, layer.topk_w, layer.ysh, out)
+
+    def fused():
+        abi.moe_ep_scatter(layer.row_of, layer.topk_w.view(torch.int32), row_gate[:T * K].view(torch.int32))
+        abi.fp8_grouped_gemm_blockscaled_combine(E + 1, layer.offsets_all, M, H, I, layer.actq, layer.acts, qw.w2,
+                                                 qw.s2, layer.rows_tok, row_gate, acc, st)
+        abi.moe_combine_finish(acc, out, None, True)
+
+    res = {"workload": "W2 + combine of the DSV3 step (T=4096, 257 groups, 36864 rows): bf16 rows stored and "
+                       "combined vs combine in the W2 epilogue (fp32 L2 reductions) + bf16 finish", "iters": iters}
+    for name, fn in (("stored_ms", stored), ("fused_ms", fused)):
+        fn()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record()
+        for _ in range(iters):
+            fn()
+        ev[1].record()
+        torch.cuda.synchronize()
+        res[name] = round(ev[0].elapsed_time(ev[1]) / iters, 4)
+    res["device_status"] = int(st.item())
+    return res
+
+
 def run_workloads(qw, pk, pk_kind, offsets_all=None, layer=None) -> dict:
     """The other configurations of the layer, each timed with CUDA events only:
     prefill with skewed routing, decode, and the dense GEMM sweep's largest
@@ -616,8 +659,9 @@ def run_workloads(qw, pk, pk_kind, offsets_all=None, layer=None) -> dict:
     out = {"gemm_dense": dense, "prefill_skew": leg_prefill(qw, pk), "decode": leg_decode(qw, pk)}
     if offsets_all is not None:
         out["wgrad"] = leg_wgrad(offsets_all, pk)
-    if layer is not None and not layer.gather:
+    if layer is not None and not layer.gather and not layer.fused_combine:
         out["gather"] = leg_gather(layer, pk)
+        out["combine"] = leg_combine(layer, pk)
     torch.cuda.empty_cache()
     return out
 

@@ -72,6 +72,7 @@ enum moe_epilogue {
     MOE_EPI_BF16 = 0,          /* C bf16 [M, N]                                      */
     MOE_EPI_F32 = 1,           /* C fp32 [M, N]                                      */
     MOE_EPI_SWIGLU_REQUANT = 2, /* N = 2I: C e4m3 [M, I] codes, sC fp32 [M, I/128]     */
+    MOE_EPI_COMBINE_F32 = 3,   /* fp8_grouped_gemm_blockscaled_combine only              */
     /* OR-ed into `epilogue`: the tile mode.  Default (neither bit) and
      * MOE_GEMM_SINGLE_CTA: one-SM tiles of 128 rows.  MOE_GEMM_PAIR_CTA: tiles
      * of 256 rows on a cluster of two SMs (tcgen05 cta_group::2), each SM
@@ -236,6 +237,34 @@ int fp8_grouped_gemm_blockscaled_gather(int32_t G, const int32_t *group_offsets,
                                         int64_t a_rows, const int32_t *a_map, const uint8_t *B,
                                         const float *sB, int32_t epilogue, void *C, float *sC,
                                         int32_t *status, void *stream);
+
+/* fp8_grouped_gemm_blockscaled with the gated combine in its epilogue
+ * ([report-walkthrough] section 3.2: y = sum_j gate_j * ffn_j(h), plus the
+ * shared expert; section 4.1: combine after the expert MLP).  Row m of group g
+ * is not stored: its bf16-rounded value, times row_gate[m], is added into the
+ * fp32 row row_token[m] of out_f32:
+ *   out_f32[row_token[m], n] += row_gate[m] * bf16(C[m, n])
+ * (C[m, n] as fp8_grouped_gemm_blockscaled defines it).  In the layer,
+ * row_token is tok_of followed by 0..T-1 and row_gate the gates in row order
+ * followed by 1 for the shared expert's rows, so out_f32 (zeroed before)
+ * receives the layer's output before its bf16 rounding; moe_combine_finish
+ * rounds it and re-zeroes the accumulator.
+ *   row_token int32 [m_capacity] (entries outside [0, out_rows) of rows in a
+ *   group raise MOE_FLAG_BAD_INDEX and that row is skipped), row_gate fp32
+ *   [m_capacity], out_f32 fp32 [out_rows, N] (16-byte aligned).
+ * The additions are fp32 reductions at the L2 in no fixed order: results agree
+ * with a fixed-order fp32 sum within its rounding bound, not bit for bit.
+ * Single tiles; other arguments and limits as fp8_grouped_gemm_blockscaled.  */
+int fp8_grouped_gemm_blockscaled_combine(int32_t G, const int32_t *group_offsets, int64_t m_capacity,
+                                         int64_t N, int64_t K, const uint8_t *A, const float *sA,
+                                         const uint8_t *B, const float *sB, const int32_t *row_token,
+                                         const float *row_gate, int64_t out_rows, float *out_f32,
+                                         int32_t *status, void *stream);
+
+/* out_bf16[i] = bf16(acc[i]) (round to nearest even) for n fp32 values (n % 8
+ * == 0, 16-byte aligned buffers); out_f32 (or NULL) receives a copy of acc;
+ * with zero != 0 acc is then set to 0 (ready for the next accumulation).    */
+int moe_combine_finish(float *acc, int64_t n, void *out_bf16, float *out_f32, int32_t zero, void *stream);
 
 /* Backward pass, weight gradient of the grouped expert GEMMs in FP8 ([repro-guide]
  * section 3: gemm_wgrad in e4m3 with 1x128 input tiles; [infra-answer]: E4M3

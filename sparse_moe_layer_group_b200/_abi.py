@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TOO_LARGE = range(6)
 MOE_FLAG_NONFINITE, MOE_FLAG_BAD_INDEX, MOE_FLAG_TIMEOUT, MOE_FLAG_BAD_OFFSETS = 1, 2, 4, 8
-MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_REQUANT = 0, 1, 2
+MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_REQUANT, MOE_EPI_COMBINE_F32 = 0, 1, 2, 3
 MOE_GEMM_SINGLE_CTA, MOE_GEMM_PAIR_CTA = 0x100, 0x200
 MOE_EP_CYCLIC, MOE_EP_BLOCK = 0, 1
 
@@ -76,6 +76,9 @@ _SIGS = {
                                                     _P, _P, _P, _P]),
     "fp8_grouped_gemm_blockscaled_gather": (ctypes.c_int, [_I32, _P, _I64, _I64, _I64, _P, _P, _I64, _P, _P, _P,
                                                            _I32, _P, _P, _P, _P]),
+    "fp8_grouped_gemm_blockscaled_combine": (ctypes.c_int, [_I32, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P,
+                                                            _I64, _P, _P, _P]),
+    "moe_combine_finish": (ctypes.c_int, [_P, _I64, _P, _P, _I32, _P]),
     "swiglu_requant": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P]),
     "fp8_quant_128x1_grouped": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _P, _I64, _P, _I64, _P, _P]),
     "fp8_grouped_gemm_wgrad": (ctypes.c_int, [_I32, _P, _I64, _I64, _I64, _P, _P, _P, _P, _I64, _I64, _P, _P,
@@ -215,6 +218,19 @@ def fp8_grouped_gemm_blockscaled_gather(G, group_offsets, m_capacity, N, K, A, s
     _check("fp8_grouped_gemm_blockscaled_gather", _lib.fp8_grouped_gemm_blockscaled_gather(
         int(G), _ptr(group_offsets), int(m_capacity), int(N), int(K), _ptr(A), _ptr(sA), int(A.shape[0]),
         _ptr(a_map), _ptr(B), _ptr(sB), int(epilogue), _ptr(C), _ptr(sC), _ptr(status), _stream(stream)))
+
+
+def fp8_grouped_gemm_blockscaled_combine(G, group_offsets, m_capacity, N, K, A, sA, B, sB, row_token, row_gate,
+                                         out_f32, status=None, stream=None):
+    """out_f32[row_token[m], :] += row_gate[m] * bf16(row m of the GEMM), fp32 [out_rows, N]."""
+    _check("fp8_grouped_gemm_blockscaled_combine", _lib.fp8_grouped_gemm_blockscaled_combine(
+        int(G), _ptr(group_offsets), int(m_capacity), int(N), int(K), _ptr(A), _ptr(sA), _ptr(B), _ptr(sB),
+        _ptr(row_token), _ptr(row_gate), int(out_f32.shape[0]), _ptr(out_f32), _ptr(status), _stream(stream)))
+
+
+def moe_combine_finish(acc, out_bf16, out_f32=None, zero: bool = True, stream=None):
+    _check("moe_combine_finish", _lib.moe_combine_finish(_ptr(acc), acc.numel(), _ptr(out_bf16), _ptr(out_f32),
+                                                         1 if zero else 0, _stream(stream)))
 
 
 def wgrad_capacities(M: int, G: int) -> tuple:

@@ -63,6 +63,24 @@ __global__ void __launch_bounds__(128) combine_kernel(const uint4 *__restrict__ 
     }
 }
 
+// 8 values per thread: two 16-byte loads, one 16-byte bf16 store.
+__global__ void combine_finish_kernel(float4 *__restrict__ acc, uint4 *__restrict__ out, float4 *__restrict__ f32,
+                                      int64_t n8, int zero) {
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= n8) return;
+    const float4 a = acc[2 * i], b = acc[2 * i + 1];
+    const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    out[i] = bf16x8(f);
+    if (f32) {
+        f32[2 * i] = a;
+        f32[2 * i + 1] = b;
+    }
+    if (zero) {
+        acc[2 * i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        acc[2 * i + 1] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+}
+
 __global__ void bias_update_kernel(int E, int64_t TK, float gamma, const int32_t *__restrict__ load,
                                    float *__restrict__ bias) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
@@ -96,5 +114,18 @@ MOE_API int moe_bias_update(int32_t E, int64_t T, int32_t K, float gamma, const 
     if (E <= 0 || T < 0 || K <= 0) return MOE_ERR_INVALID_ARG;
     if (!expert_load || !e_bias) return MOE_ERR_INVALID_ARG;
     bias_update_kernel<<<(E + 255) / 256, 256, 0, as_stream(stream)>>>(E, T * K, gamma, expert_load, e_bias);
+    return launch_status();
+}
+
+MOE_API int moe_combine_finish(float *acc, int64_t n, void *out_bf16, float *out_f32, int32_t zero, void *stream) {
+    if (n < 0 || n % 8 != 0) return MOE_ERR_INVALID_ARG;
+    if (n == 0) return MOE_OK;
+    if (!acc || !out_bf16 || !aligned16(acc) || !aligned16(out_bf16) || (out_f32 && !aligned16(out_f32)))
+        return MOE_ERR_INVALID_ARG;
+    const int64_t n8 = n / 8;
+    if ((n8 + 255) / 256 > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+    combine_finish_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, as_stream(stream)>>>(
+        reinterpret_cast<float4 *>(acc), static_cast<uint4 *>(out_bf16), reinterpret_cast<float4 *>(out_f32), n8,
+        zero ? 1 : 0);
     return launch_status();
 }

@@ -49,6 +49,14 @@
 // outside the group read source row 0 (computed, never stored).  The epilogue
 // reads the A row scales through the same map.
 //
+// Combine variant (template parameter COMBINE, single tiles, the W2 GEMM of the
+// layer): instead of storing row m, the epilogue adds c_gate[m] * bf16(C[m, :])
+// into the fp32 row c_tok[m] of an output accumulator with vector reductions at
+// the L2 (red.global.add.v4.f32): the gated combine of the routed rows (and, with
+// gate 1, of the shared expert's rows) happens inside the GEMM, and the permuted
+// rows are never written.  The additions to one output row come from different
+// CTAs in no fixed order, so the fp32 sums are not reproducible bit for bit.
+//
 // No TMA multicast: every CTA loads its own tiles.  Every work wait is bounded
 // (by default 2 s, see wait_limit_ns); on expiry the CTA raises MOE_FLAG_TIMEOUT,
 // drains its own outstanding TMA loads and MMAs (waits of up to 2 s each), frees
@@ -166,15 +174,17 @@ __device__ __forceinline__ int remap_tile(int v, int R, int S, int C) {
     return v;
 }
 
-template <bool PAIR, bool GATHER>
+template <bool PAIR, bool GATHER, bool COMBINE>
 __global__ void __launch_bounds__(THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC,
                     const int32_t *__restrict__ offs, int G, int64_t m_cap, int N, int K,
                     const float *__restrict__ sA, const float *__restrict__ sB, int epi,
                     void *__restrict__ C, float *__restrict__ sC, int32_t *status, uint64_t wait_ns,
-                    int stall, const int32_t *__restrict__ a_map, int64_t a_rows) {
+                    int stall, const int32_t *__restrict__ a_map, int64_t a_rows,
+                    const int32_t *__restrict__ c_tok, const float *__restrict__ c_gate, int64_t c_rows) {
     static_assert(!(PAIR && GATHER), "the gather variant runs single tiles");
+    static_assert(!(PAIR && COMBINE), "the combine variant runs single tiles");
     using Cf = Cfg<PAIR>;
     constexpr int STAGES = Cf::STAGES;
     constexpr uint32_t STAGE_BYTES = Cf::STAGE_BYTES;
@@ -470,7 +480,28 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const bool full_warp = nvalid == 32;
             if (lane == 0) bulk_wait_read();
             __syncwarp();
-            if (!swiglu) {
+            if (COMBINE) {
+                // the gated row, bf16-rounded as a stored expert row would be, added into
+                // its token's fp32 output row
+                const int64_t n0 = static_cast<int64_t>(tl.nt) * BN + 128 * half;
+                if (n0 < N && store_row) {
+                    const int tok = __ldg(c_tok + grow);
+                    const float gate = __ldg(c_gate + grow);
+                    if (tok >= 0 && tok < c_rows) {
+                        float *dst = reinterpret_cast<float *>(C) + static_cast<int64_t>(tok) * N + n0;
+#pragma unroll
+                        for (int j = 0; j < 128; j += 4) {
+                            float v[4];
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                v[q] = __fmul_rn(gate, __bfloat162float(__float2bfloat16_rn(acc[j + q])));
+                            red_add_f32x4(dst + j, v[0], v[1], v[2], v[3]);
+                        }
+                    } else {
+                        set_flag(status, MOE_FLAG_BAD_INDEX);
+                    }
+                }
+            } else if (!swiglu) {
                 const int64_t n0 = static_cast<int64_t>(tl.nt) * BN + 128 * half;
                 if (n0 < N) {
                     if (epi == MOE_EPI_BF16) {
@@ -608,17 +639,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
 // Once per device and kernel variant: check the register split and raise the
 // dynamic shared-memory limit.  Returns a moe_status.
-template <bool PAIR, bool GATHER>
+template <bool PAIR, bool GATHER, bool COMBINE>
 static int prepare_kernel() {
     static int state[MAX_DEVICES] = {};
     static std::mutex mu;
     const int r = once_per_device(state, mu, []() {
         cudaFuncAttributes attr;
-        if (cudaFuncGetAttributes(&attr, grouped_gemm_kernel<PAIR, GATHER>) != cudaSuccess) return -MOE_ERR_CUDA;
+        if (cudaFuncGetAttributes(&attr, grouped_gemm_kernel<PAIR, GATHER, COMBINE>) != cudaSuccess)
+            return -MOE_ERR_CUDA;
         // setmaxnreg moves registers inside the launch's allotment: the split
         // 128 x 40 + 256 x 232 must equal 384 x (registers at launch)
         if (attr.numRegs != LAUNCH_REGS) return -MOE_ERR_UNSUPPORTED;
-        if (cudaFuncSetAttribute(grouped_gemm_kernel<PAIR, GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(grouped_gemm_kernel<PAIR, GATHER, COMBINE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(Cfg<PAIR>::SMEM_BYTES)) != cudaSuccess)
             return -MOE_ERR_CUDA;
         return 1;
@@ -643,7 +675,7 @@ static int pair_clusters() {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<true, false>, &cfg) == cudaSuccess && n > 0)
+        if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<true, false, false>, &cfg) == cudaSuccess && n > 0)
             return n;
         return num_sms() / 2;
     });
@@ -654,21 +686,29 @@ static int pair_clusters() {
 // a_map[m] (gather variant, single tiles).
 static int grouped_gemm(int32_t G, const int32_t *group_offsets, int64_t m_capacity, int64_t N, int64_t K,
                         const uint8_t *A, const float *sA, const int32_t *a_map, int64_t a_rows, const uint8_t *B,
-                        const float *sB, int32_t epilogue, void *C, float *sC, int32_t *status, void *stream) {
+                        const float *sB, int32_t epilogue, void *C, float *sC, int32_t *status, void *stream,
+                        const int32_t *c_tok = nullptr, const float *c_gate = nullptr, int64_t c_rows = 0) {
     const bool gather = a_map != nullptr;
+    const bool combine = c_tok != nullptr;
+    if (gather && combine) return MOE_ERR_UNSUPPORTED;
     // tile mode: one-SM tiles unless CTA pairs are asked for (measured on B200:
     // pairs are 25 % slower at 128 tokens per expert, where 256-row tiles are
     // mostly padding, and about 1 % faster at 1024 tokens per expert)
-    const bool single = gather || (epilogue & MOE_GEMM_PAIR_CTA) == 0 || (epilogue & MOE_GEMM_SINGLE_CTA) != 0;
+    const bool single = gather || combine || (epilogue & MOE_GEMM_PAIR_CTA) == 0 ||
+                        (epilogue & MOE_GEMM_SINGLE_CTA) != 0;
     epilogue &= ~(MOE_GEMM_SINGLE_CTA | MOE_GEMM_PAIR_CTA);
-    if (G < 0 || m_capacity < 0 || N < 0 || K < 0 || a_rows < 0) return MOE_ERR_INVALID_ARG;
+    if (G < 0 || m_capacity < 0 || N < 0 || K < 0 || a_rows < 0 || c_rows < 0) return MOE_ERR_INVALID_ARG;
     if (N % 128 != 0 || K % 128 != 0) return MOE_ERR_INVALID_ARG;
-    if (epilogue != MOE_EPI_BF16 && epilogue != MOE_EPI_F32 && epilogue != MOE_EPI_SWIGLU_REQUANT)
+    if (combine ? epilogue != MOE_EPI_COMBINE_F32
+                : (epilogue != MOE_EPI_BF16 && epilogue != MOE_EPI_F32 && epilogue != MOE_EPI_SWIGLU_REQUANT))
         return MOE_ERR_INVALID_ARG;
     if (epilogue == MOE_EPI_SWIGLU_REQUANT && (N % 256 != 0 || !sC)) return MOE_ERR_INVALID_ARG;
     if (G == 0 || m_capacity == 0 || N == 0) return MOE_OK;
     if (K == 0) return MOE_ERR_UNSUPPORTED;   // an empty reduction is not a GEMM this kernel runs
     if (gather && a_rows == 0) return MOE_ERR_INVALID_ARG;
+    if (combine && (c_rows == 0 || !c_gate || (reinterpret_cast<uintptr_t>(c_tok) & 3) ||
+                    (reinterpret_cast<uintptr_t>(c_gate) & 3) || c_rows > 0x7fffffffLL))
+        return MOE_ERR_INVALID_ARG;
     const int max_groups = single ? Cfg<false>::MAX_GROUPS : Cfg<true>::MAX_GROUPS;
     if (G > max_groups || m_capacity > 0x7fffffffLL || N > 0x7fffffffLL || K > 0x7fffffffLL ||
         a_rows > 0x7fffffffLL)
@@ -678,8 +718,9 @@ static int grouped_gemm(int32_t G, const int32_t *group_offsets, int64_t m_capac
         (reinterpret_cast<uintptr_t>(sB) & 3) || (sC && (reinterpret_cast<uintptr_t>(sC) & 3)) ||
         (reinterpret_cast<uintptr_t>(a_map) & 3))
         return MOE_ERR_INVALID_ARG;
-    int rc = gather ? prepare_kernel<false, true>() : single ? prepare_kernel<false, false>()
-                                                              : prepare_kernel<true, false>();
+    int rc = gather ? prepare_kernel<false, true, false>()
+             : combine ? prepare_kernel<false, false, true>()
+             : single ? prepare_kernel<false, false, false>() : prepare_kernel<true, false, false>();
     if (rc != MOE_OK) return rc;
     auto enc = encode_fn();
     if (!enc) return MOE_ERR_CUDA;
@@ -724,8 +765,8 @@ static int grouped_gemm(int32_t G, const int32_t *group_offsets, int64_t m_capac
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return MOE_ERR_CUDA;
     }
-    if (epilogue == MOE_EPI_F32) {
-        tmC = tmA;
+    if (epilogue == MOE_EPI_F32 || epilogue == MOE_EPI_COMBINE_F32) {
+        tmC = tmA;   // unused: these epilogues write without TMA
     } else {
         const bool codes = epilogue == MOE_EPI_SWIGLU_REQUANT;
         const int64_t cols = codes ? N / 2 : N;
@@ -744,15 +785,21 @@ static int grouped_gemm(int32_t G, const int32_t *group_offsets, int64_t m_capac
     const uint64_t wait_ns = wait_limit_ns();
     const int stall = test_stall() ? 1 : 0;
     if (gather) {
-        grouped_gemm_kernel<false, true><<<num_sms(), THREADS, Cfg<false>::smem_bytes(G), st>>>(
+        grouped_gemm_kernel<false, true, false><<<num_sms(), THREADS, Cfg<false>::smem_bytes(G), st>>>(
             tmA, tmB, tmC, group_offsets, G, m_capacity, n, k, sA, sB, epilogue, C, sC, status, wait_ns, stall,
-            a_map, a_rows);
+            a_map, a_rows, nullptr, nullptr, 0);
+        return launch_status();
+    }
+    if (combine) {
+        grouped_gemm_kernel<false, false, true><<<num_sms(), THREADS, Cfg<false>::smem_bytes(G), st>>>(
+            tmA, tmB, tmC, group_offsets, G, m_capacity, n, k, sA, sB, epilogue, C, sC, status, wait_ns, stall,
+            nullptr, 0, c_tok, c_gate, c_rows);
         return launch_status();
     }
     if (single) {
-        grouped_gemm_kernel<false, false><<<num_sms(), THREADS, Cfg<false>::smem_bytes(G), st>>>(
+        grouped_gemm_kernel<false, false, false><<<num_sms(), THREADS, Cfg<false>::smem_bytes(G), st>>>(
             tmA, tmB, tmC, group_offsets, G, m_capacity, n, k, sA, sB, epilogue, C, sC, status, wait_ns, stall,
-            nullptr, 0);
+            nullptr, 0, nullptr, nullptr, 0);
         return launch_status();
     }
     cudaLaunchConfig_t cfg = {};
@@ -767,9 +814,11 @@ static int grouped_gemm(int32_t G, const int32_t *group_offsets, int64_t m_capac
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<true, false>, tmA, tmB, tmC, group_offsets, G, m_capacity, n, k,
-                           sA, sB, static_cast<int>(epilogue), C, sC, status, wait_ns, 0,
-                           static_cast<const int32_t *>(nullptr), static_cast<int64_t>(0)) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<true, false, false>, tmA, tmB, tmC, group_offsets, G, m_capacity,
+                           n, k, sA, sB, static_cast<int>(epilogue), C, sC, status, wait_ns, 0,
+                           static_cast<const int32_t *>(nullptr), static_cast<int64_t>(0),
+                           static_cast<const int32_t *>(nullptr), static_cast<const float *>(nullptr),
+                           static_cast<int64_t>(0)) != cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_status();
 }
@@ -795,4 +844,14 @@ MOE_API int fp8_grouped_gemm_blockscaled_gather(int32_t G, const int32_t *group_
     if (!a_map) return MOE_ERR_INVALID_ARG;
     return gg::grouped_gemm(G, group_offsets, m_capacity, N, K, A, sA, a_map, a_rows, B, sB, epilogue, C, sC, status,
                             stream);
+}
+
+MOE_API int fp8_grouped_gemm_blockscaled_combine(int32_t G, const int32_t *group_offsets, int64_t m_capacity,
+                                                 int64_t N, int64_t K, const uint8_t *A, const float *sA,
+                                                 const uint8_t *B, const float *sB, const int32_t *row_token,
+                                                 const float *row_gate, int64_t out_rows, float *out_f32,
+                                                 int32_t *status, void *stream) {
+    if (!row_token) return MOE_ERR_INVALID_ARG;
+    return gg::grouped_gemm(G, group_offsets, m_capacity, N, K, A, sA, nullptr, 0, B, sB, MOE_EPI_COMBINE_F32,
+                            out_f32, nullptr, status, stream, row_token, row_gate, out_rows);
 }

@@ -109,6 +109,14 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *tm,
         : "memory");
 }
 
+// Four fp32 additions into global memory, performed at the L2 (no return value).
+// The address is 16-byte aligned.  The order of concurrent additions to one
+// address is unspecified.
+__device__ __forceinline__ void red_add_f32x4(float *p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
 // Plain (untiled) bulk copy global -> this CTA's shared memory, completing on
 // an mbarrier; both addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,

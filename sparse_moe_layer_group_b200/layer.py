@@ -20,7 +20,11 @@ the forward runs in the library's kernels:
                       shape (32 four-row gathers per A tile instead of one
                       tiled load), hence not the default
   5  grouped GEMM     W2 of the same E + 1 groups -> bf16 rows
-  6  moe_combine      gate-weighted sum of the K rows + the shared row -> bf16
+  6  moe_combine      gate-weighted sum of the K rows + the shared row -> bf16.
+                      With fused_combine=True the W2 GEMM adds each gated row
+                      into an fp32 accumulator of the output itself (no rows
+                      stored; additions in no fixed order) and
+                      moe_combine_finish rounds it to bf16
   (7 moe_bias_update  after the step, from the expert loads of step 3)
 
 Treating the shared expert as one more group of the same two launches lets its
@@ -89,10 +93,12 @@ class MoELayer:
 
     def __init__(self, T: int, H: int, E: int, K: int, n_group: int, topk_group: int, I: int,
                  rho: float, w_router: torch.Tensor, e_bias: torch.Tensor, weights: QuantWeights,
-                 router_offset: Optional[torch.Tensor] = None, device="cuda", gather: bool = False):
+                 router_offset: Optional[torch.Tensor] = None, device="cuda", gather: bool = False,
+                 fused_combine: bool = False):
         self.T, self.H, self.E, self.K, self.I = T, H, E, K, I
-        self.gather = gather
-        self.launches_per_forward = LAUNCHES_PER_FORWARD - (1 if gather else 0)
+        self.gather, self.fused_combine = gather, fused_combine
+        # the fused combine adds a gate scatter and a finishing pass and drops the combine kernel
+        self.launches_per_forward = LAUNCHES_PER_FORWARD - (1 if gather else 0) + (1 if fused_combine else 0)
         self.n_group, self.topk_group, self.rho = n_group, topk_group, rho
         self.d = abi.dims(T, H, E, K, n_group, topk_group, I, rho)
         self.w_router, self.e_bias, self.router_offset = w_router, e_bias, router_offset
@@ -115,14 +121,16 @@ class MoELayer:
         self.ws = torch.empty((ws_bytes + 255) // 256 * 256, **u8)
         # rows of the first GEMM: rows 0..T*K-1 the routed (token, slot) pairs in
         # expert order, rows T*K..T*K+T-1 the tokens themselves (shared expert)
+        # token of every row: tok_of (written by moe_permute), then 0..T-1
+        self.rows_tok = torch.empty(TK + T, **i32)
+        self.rows_tok[TK:] = torch.arange(T, **i32)
+        self.tok_of = self.rows_tok[:TK]
         if gather:
-            # read through a_map = (tok_of, 0..T-1) from the T quantised token rows
+            # read through rows_tok from the T quantised token rows
             self.aq = self.as_ = None
             self.xq = torch.empty(T, H, **u8)
             self.xs = torch.empty(T, H // 128, **f32)
-            self.a_map = torch.empty(TK + T, **i32)
-            self.a_map[TK:] = torch.arange(T, **i32)
-            self.tok_of = self.a_map[:TK]
+            self.a_map = self.rows_tok
         else:
             # a materialised copy in that order; the last T rows are the quantiser's output
             self.aq = torch.empty(TK + T, H, **u8)
@@ -130,7 +138,6 @@ class MoELayer:
             self.xq = self.aq[TK:]
             self.xs = self.as_[TK:]
             self.a_map = None
-            self.tok_of = torch.empty(TK, **i32)
         self.load = torch.empty(E, **i32)
         # group offsets of the E + 1 groups: moe_permute writes entries 0..E,
         # entry E + 1 closes the shared group
@@ -139,8 +146,15 @@ class MoELayer:
         self.row_of = torch.empty(TK, **i32)
         self.actq = torch.empty(TK + T, I, **u8)
         self.acts = torch.empty(TK + T, I // 128, **f32)
-        self.yperm = torch.empty(TK + T, H, **bf)
-        self.ysh = self.yperm[TK:]
+        if fused_combine:
+            # gate of every row in row order (1 for the shared expert's rows) and the
+            # fp32 accumulator of the output (zero between forwards)
+            self.row_gate = torch.ones(TK + T, **f32)
+            self.out_acc = torch.zeros(T, H, **f32)
+            self.yperm = self.ysh = None
+        else:
+            self.yperm = torch.empty(TK + T, H, **bf)
+            self.ysh = self.yperm[TK:]
         self.out = torch.empty(T, H, **bf)
         self.out_f32 = None
         self.status = torch.zeros(1, **i32)
@@ -188,6 +202,17 @@ class MoELayer:
                                              qw.s13, abi.MOE_EPI_SWIGLU_REQUANT, self.actq, self.acts, st, stream)
         if gemm_events is not None:
             gemm_events[1].record(ev_stream)
+        if self.fused_combine:
+            # the gates into row order (fp32 moved as its bit pattern), then W2 adds
+            # every gated row into the output accumulator
+            abi.moe_ep_scatter(self.row_of, self.topk_w.view(torch.int32), self.row_gate[:T * K].view(torch.int32),
+                               stream)
+            abi.fp8_grouped_gemm_blockscaled_combine(E + 1, self.offsets_all, M, H, I, self.actq, self.acts, qw.w2,
+                                                     qw.s2, self.rows_tok, self.row_gate, self.out_acc, st, stream)
+            if gemm_events is not None:
+                gemm_events[2].record(ev_stream)
+            abi.moe_combine_finish(self.out_acc, out, self.out_f32 if out_f32 else None, True, stream)
+            return out
         abi.fp8_grouped_gemm_blockscaled(E + 1, self.offsets_all, M, H, I, self.actq, self.acts, qw.w2, qw.s2,
                                          abi.MOE_EPI_BF16, self.yperm, None, st, stream)
         if gemm_events is not None:
@@ -200,8 +225,8 @@ class MoELayer:
         """The header's moe_layer for this layer's buffers (the materialised
         path), for moe_layer_forward / moe_layer_run_host: the whole forward,
         and the bias update into bias_out if given, behind one C call."""
-        if self.gather:
-            raise ValueError("the one-call forward runs the materialised path (gather=False)")
+        if self.gather or self.fused_combine:
+            raise ValueError("the one-call forward runs the materialised path (gather=False, fused_combine=False)")
         qw = self.qw
         bufs = dict(w13=qw.w13, s13=qw.s13, w2=qw.w2, s2=qw.s2, w_pieces=self.w_pieces, e_bias=self.e_bias,
                     router_offset=self.router_offset, topk_idx=self.topk_idx, topk_w=self.topk_w,
