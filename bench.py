@@ -430,7 +430,7 @@ def leg_prefill(qw, pk, steps: int = 20) -> dict:
 
 def leg_decode(qw, pk, steps: int = 50) -> dict:
     """Decode-sized batch: T = 128 tokens at the DeepSeek-V3 shape, all 257
-    experts' E4M3 weights resident; judged by the HBM bandwidth of the expert
+    experts' E4M3 weights resident; measured against the HBM bandwidth of the expert
     weights the step actually touches (every expert with a routed token, plus
     the shared expert), read by the two grouped GEMMs."""
     s = synth.DECODE

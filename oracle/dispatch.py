@@ -75,7 +75,8 @@ def combine_by_rank(yperm, row_of, w, rank, yshared=None):
     selected; section 4.1 has the node compute the token's experts there and
     accumulate their results while the combine forwards them back.  Each rank's
     gated partial sum is the row that crosses back; it is stored in bf16, the
-    precision of the expert rows it sums (R12), and the source adds the partials.
+    precision in which the layer stores the expert rows it sums, and the source
+    adds the partials.
     rank int [T, K]: the rank of each slot's expert."""
     w64 = np.asarray(w, dtype=np.float64)
     T, K = w64.shape
