@@ -501,6 +501,91 @@ def leg_gemm_dense(pk, M: int = 4096, N: int = 18432, K: int = 7168, iters: int 
             "l2": "flushed before every launch (256 MB write)"}
 
 
+def leg_gemm_sweep(pk, qw, iters: int = 10) -> list:
+    """The FP8 block-scaled GEMM sweep: dense C = A B^T for (N, K) in {(4096, 7168),
+    (7168, 2048), (18432, 7168), (7168, 18432)} and M in {128, 1024, 4096, 16384}
+    (A N(0,1) with 1 % of the entries x100, B N(0, 0.02)), and 256-group GEMMs on
+    the layer's own resident expert weights (W13: N=4096, K=7168; W2: N=7168,
+    K=2048) with 8M rows split by a seeded uniform random composition (sorted
+    uniform cut points, empty groups allowed).  Each launch timed alone after a
+    256 MB L2 flush, median of `iters`; TFLOP/s against 2 x the measured bf16
+    burst and algorithmic bytes (A, B and scales read, C written) against the
+    HBM copy peak."""
+    import sparse_moe_layer_group_b200 as moe
+    abi = moe.abi
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    peak = 2.0 * pk["bf16_tflops"]
+
+    def timed(run):
+        for _ in range(2):
+            run()
+        t = []
+        for _ in range(iters):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            run()
+            e1.record()
+            e1.synchronize()
+            t.append(e0.elapsed_time(e1))
+        return statistics.median(t)
+
+    def row(kind, M, N, K, G, ms, nbytes):
+        fl = 2 * M * N * K
+        return {"kind": kind, "M": M, "N": N, "K": K, "groups": G, "ms": round(ms, 4),
+                "tflops": round(fl / ms / 1e9, 1), "frac_of_fp8_peak": round(fl / ms / 1e9 / peak, 3),
+                "gbs": round(nbytes / ms / 1e6, 1), "frac_of_hbm": round(nbytes / ms / 1e6 / pk["hbm_gbs"], 3)}
+
+    out = []
+    Ms = (128, 1024, 4096, 16384)
+    for N, K in ((4096, 7168), (7168, 2048), (18432, 7168), (7168, 18432)):
+        b = synth.normal((N, K), 0.02, 72, device="cuda", dtype=torch.bfloat16)
+        qb = torch.empty(1, N, K, dtype=torch.uint8, device="cuda")
+        sb = torch.empty(1, N // 128, K // 128, dtype=torch.float32, device="cuda")
+        abi.fp8_quant_128x128(b, qb[0], sb[0])
+        del b
+        for M in Ms:
+            a = synth.heavy_tailed(M, K, 71, device="cuda")
+            qa = torch.empty(M, K, dtype=torch.uint8, device="cuda")
+            sa = torch.empty(M, K // 128, dtype=torch.float32, device="cuda")
+            abi.fp8_quant_1x128(a, qa, sa)
+            del a
+            C = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+            offs = torch.tensor([0, M], dtype=torch.int32, device="cuda")
+            ms = timed(lambda: abi.fp8_grouped_gemm_blockscaled(1, offs, M, N, K, qa, sa, qb, sb, abi.MOE_EPI_BF16,
+                                                                C))
+            nbytes = M * K + N * K + M * (K // 128) * 4 + (N // 128) * (K // 128) * 4 + 2 * M * N
+            out.append(row("dense", M, N, K, 1, ms, nbytes))
+            del qa, sa, C
+        del qb, sb
+    # 256 groups on the resident expert weights, 8M rows in a seeded random composition
+    G = 256
+    for name, W, S, N, K in (("W13", qw.w13, qw.s13, qw.w13.shape[1], qw.w13.shape[2]),
+                             ("W2", qw.w2, qw.s2, qw.w2.shape[1], qw.w2.shape[2])):
+        for M in Ms[:3]:
+            rows = 8 * M
+            g = synth.gen(900 + M, "cpu")
+            cuts = torch.sort(torch.randint(0, rows + 1, (G - 1,), generator=g)).values
+            offs_h = torch.cat([torch.zeros(1, dtype=torch.int64), cuts, torch.tensor([rows])])
+            offs = offs_h.to(torch.int32).cuda()
+            a = synth.heavy_tailed(rows, K, 73, device="cuda")
+            qa = torch.empty(rows, K, dtype=torch.uint8, device="cuda")
+            sa = torch.empty(rows, K // 128, dtype=torch.float32, device="cuda")
+            abi.fp8_quant_1x128(a, qa, sa)
+            del a
+            C = torch.empty(rows, N, dtype=torch.bfloat16, device="cuda")
+            ms = timed(lambda: abi.fp8_grouped_gemm_blockscaled(G, offs, rows, N, K, qa, sa, W, S, abi.MOE_EPI_BF16,
+                                                                C))
+            touched = int(((offs_h[1:] - offs_h[:-1]) > 0).sum())
+            nbytes = (rows * K + touched * (N * K + (N // 128) * (K // 128) * 4) + rows * (K // 128) * 4
+                      + 2 * rows * N)
+            out.append(row(f"grouped {name}", rows, N, K, G, ms, nbytes))
+            del qa, sa, C
+    del flush
+    torch.cuda.empty_cache()
+    return out
+
+
 def leg_wgrad(offsets_all, pk, iters: int = 5) -> dict:
     """Backward weight gradient of W13 at the DeepSeek-V3 layer shape: dW13 [257,
     2I, H] = dY^T X per expert over the layer's own expert segments (the T*K
@@ -656,7 +741,10 @@ def run_workloads(qw, pk, pk_kind, offsets_all=None, layer=None) -> dict:
     with ClockSampler(torch.cuda.current_device()) as clk:
         dense = leg_gemm_dense(pk)
     dense["clocks"] = clk.summary()
-    out = {"gemm_dense": dense, "prefill_skew": leg_prefill(qw, pk), "decode": leg_decode(qw, pk)}
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        sweep = leg_gemm_sweep(pk, qw)
+    out = {"gemm_dense": dense, "gemm_sweep": {"shapes": sweep, "clocks": clk.summary()},
+           "prefill_skew": leg_prefill(qw, pk), "decode": leg_decode(qw, pk)}
     if offsets_all is not None:
         out["wgrad"] = leg_wgrad(offsets_all, pk)
     if layer is not None and not layer.gather and not layer.fused_combine:
