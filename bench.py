@@ -504,10 +504,11 @@ def leg_gemm_dense(pk, M: int = 4096, N: int = 18432, K: int = 7168, iters: int 
 def leg_gemm_sweep(pk, qw, iters: int = 10) -> list:
     """The FP8 block-scaled GEMM sweep: dense C = A B^T for (N, K) in {(4096, 7168),
     (7168, 2048), (18432, 7168), (7168, 18432)} and M in {128, 1024, 4096, 16384}
-    (A N(0,1) with 1 % of the entries x100, B N(0, 0.02)), and 256-group GEMMs on
-    the layer's own resident expert weights (W13: N=4096, K=7168; W2: N=7168,
-    K=2048) with 8M rows split by a seeded uniform random composition (sorted
-    uniform cut points, empty groups allowed).  Each launch timed alone after a
+    (A N(0,1) with 1 % of the entries x100, B N(0, 0.02)), and each shape as a
+    256-group GEMM with 8M rows split by a seeded uniform random composition
+    (sorted uniform cut points, empty groups allowed) over 256 weight matrices
+    (the layer's resident experts for its two shapes W13 and W2, drawn N(0, 0.02)
+    for the other two).  Each launch timed alone after a
     256 MB L2 flush, median of `iters`; TFLOP/s against 2 x the measured bf16
     burst and algorithmic bytes (A, B and scales read, C written) against the
     HBM copy peak."""
@@ -558,11 +559,23 @@ def leg_gemm_sweep(pk, qw, iters: int = 10) -> list:
             out.append(row("dense", M, N, K, 1, ms, nbytes))
             del qa, sa, C
         del qb, sb
-    # 256 groups on the resident expert weights, 8M rows in a seeded random composition
+    # 256 groups, 8M rows in a seeded uniform random composition; the two layer shapes
+    # reuse the resident expert weights, the other two draw 256 weight matrices
     G = 256
-    for name, W, S, N, K in (("W13", qw.w13, qw.s13, qw.w13.shape[1], qw.w13.shape[2]),
-                             ("W2", qw.w2, qw.s2, qw.w2.shape[1], qw.w2.shape[2])):
-        for M in Ms[:3]:
+    for N, K in ((4096, 7168), (7168, 2048), (18432, 7168), (7168, 18432)):
+        if (N, K) == tuple(qw.w13.shape[1:]):
+            name, W, S = "W13", qw.w13, qw.s13
+        elif (N, K) == tuple(qw.w2.shape[1:]):
+            name, W, S = "W2", qw.w2, qw.s2
+        else:
+            name = f"{N}x{K}"
+            W = torch.empty(G, N, K, dtype=torch.uint8, device="cuda")
+            S = torch.empty(G, N // 128, K // 128, dtype=torch.float32, device="cuda")
+            for e in range(G):
+                b = synth.normal((N, K), 0.02, 1000 + e, device="cuda", dtype=torch.bfloat16)
+                abi.fp8_quant_128x128(b, W[e], S[e])
+                del b
+        for M in Ms:
             rows = 8 * M
             g = synth.gen(900 + M, "cpu")
             cuts = torch.sort(torch.randint(0, rows + 1, (G - 1,), generator=g)).values
@@ -581,6 +594,8 @@ def leg_gemm_sweep(pk, qw, iters: int = 10) -> list:
                       + 2 * rows * N)
             out.append(row(f"grouped {name}", rows, N, K, G, ms, nbytes))
             del qa, sa, C
+        del W, S
+        torch.cuda.empty_cache()
     del flush
     torch.cuda.empty_cache()
     return out
