@@ -382,8 +382,9 @@ int moe_ep_scatter_rows(const int32_t *row_of, const int32_t *values, int64_t n,
  * bf16 [T,H]) is uploaded on a stream of its own into x_dev[i % 2], the forward
  * runs on `stream` into out_dev[i % 2], and out_host[i] (pinned) is downloaded
  * on a third stream, so the copies of batches i+1 and i-1 overlap batch i's
- * forward.  One cudaMemcpyAsync per copy.  Returns once everything is enqueued;
- * `stream` completes after the last download.                                 */
+ * forward.  One cudaMemcpyAsync per copy; the copies start after the work
+ * already enqueued on `stream`.  Returns once everything is enqueued; `stream`
+ * completes after the last download.                                          */
 typedef struct {
     moe_dims dims;
     const uint8_t *w13;

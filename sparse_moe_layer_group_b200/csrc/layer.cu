@@ -50,11 +50,17 @@ MOE_API int moe_layer_run_host(const moe_layer *L, const void *const *x_host, vo
         if (!x_host[i] || !out_host[i]) return MOE_ERR_INVALID_ARG;
     const size_t bytes = static_cast<size_t>(L->dims.T) * L->dims.H * 2;
     cudaStream_t st = as_stream(stream), up = nullptr, down = nullptr;
-    cudaEvent_t in_done[2] = {}, fwd_done[2] = {}, out_done[2] = {};
+    cudaEvent_t in_done[2] = {}, fwd_done[2] = {}, out_done[2] = {}, start = nullptr;
     int rc = MOE_OK;
     auto fail = [&](int code) { rc = code; };
     if (cudaStreamCreateWithFlags(&up, cudaStreamNonBlocking) != cudaSuccess ||
         cudaStreamCreateWithFlags(&down, cudaStreamNonBlocking) != cudaSuccess)
+        fail(MOE_ERR_CUDA);
+    // the copies start after the work already on `stream` (e.g. an earlier call
+    // whose forwards still read x_dev or write out_dev)
+    if (rc == MOE_OK && (cudaEventCreateWithFlags(&start, cudaEventDisableTiming) != cudaSuccess ||
+                         cudaEventRecord(start, st) != cudaSuccess || cudaStreamWaitEvent(up, start, 0) != cudaSuccess ||
+                         cudaStreamWaitEvent(down, start, 0) != cudaSuccess))
         fail(MOE_ERR_CUDA);
     for (int b = 0; b < 2 && rc == MOE_OK; ++b)
         if (cudaEventCreateWithFlags(&in_done[b], cudaEventDisableTiming) != cudaSuccess ||
@@ -92,6 +98,7 @@ MOE_API int moe_layer_run_host(const moe_layer *L, const void *const *x_host, vo
         cudaStreamSynchronize(down);
     }
     // released once their work completes
+    if (start) cudaEventDestroy(start);
     for (int b = 0; b < 2; ++b) {
         if (in_done[b]) cudaEventDestroy(in_done[b]);
         if (fwd_done[b]) cudaEventDestroy(fwd_done[b]);

@@ -266,6 +266,11 @@ def test_layer_one_call_forward_and_host_runner(lib, shape):
     x_dev = [torch.empty_like(ref[0]) for _ in range(2)]
     out_dev = [torch.empty_like(ref[0]) for _ in range(2)]
     layer.run_host(x_host, out_host, x_dev, out_dev)
+    # a second call right behind the first, on the same device buffers: its
+    # uploads wait for the first call's forwards
+    out_host2 = [torch.full_like(o, float("nan")).pin_memory() for o in out_host]
+    layer.run_host(x_host[::-1], out_host2, x_dev, out_dev)
     torch.cuda.synchronize()
     for i in range(3):
         assert torch.equal(out_host[i], ref[i].cpu()), f"batch {i}"
+        assert torch.equal(out_host2[i], ref[2 - i].cpu()), f"second call, batch {i}"
