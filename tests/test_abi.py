@@ -84,6 +84,14 @@ def test_host_validation_rejects_before_launch():
     assert gg(1, 16, 64, 256, 128, 16, 16, 0, 16, 16, 16, 0, 16, None, None, None) == a.MOE_ERR_INVALID_ARG
     assert gg(1, 16, 64, 256, 100, 16, 16, 8, 16, 16, 16, 0, 16, None, None, None) == a.MOE_ERR_INVALID_ARG
     assert gg(0, 16, 64, 256, 128, 16, 16, 8, 16, 16, 16, 0, 16, None, None, None) == 0
+    # combine variant: token and gate maps required and 4-byte aligned, out_rows >= 1; finish n % 8 == 0
+    gc = L.fp8_grouped_gemm_blockscaled_combine
+    assert gc(1, 16, 64, 256, 128, 16, 16, 16, 16, None, 16, 8, 16, None, None) == a.MOE_ERR_INVALID_ARG
+    assert gc(1, 16, 64, 256, 128, 16, 16, 16, 16, 16, 18, 8, 16, None, None) == a.MOE_ERR_INVALID_ARG
+    assert gc(1, 16, 64, 256, 128, 16, 16, 16, 16, 16, 16, 0, 16, None, None) == a.MOE_ERR_INVALID_ARG
+    assert gc(0, 16, 64, 256, 128, 16, 16, 16, 16, 16, 16, 8, 16, None, None) == 0
+    assert L.moe_combine_finish(16, 12, 16, None, 1, None) == a.MOE_ERR_INVALID_ARG
+    assert L.moe_combine_finish(16, 0, 16, None, 1, None) == 0
     # one-call forward and host runner: the struct and buffers are required, n >= 0
     assert L.moe_layer_forward(None, 16, 16, None) == a.MOE_ERR_INVALID_ARG
     lay = a.MoeLayerC()
