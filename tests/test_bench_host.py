@@ -47,3 +47,34 @@ def test_reference_step_sampler_and_rank_split():
     assert math.isfinite(v) and v > 0
     args = argparse.Namespace(steps=1, warmup=0)
     assert bench.run_reference(args, rank=1, world=2) is None    # only rank 0 works
+
+
+def _fake_smi(tmp_path, period_s: float, mhz: int):
+    """A stand-in nvidia-smi on PATH that prints one CSV sample per period."""
+    exe = tmp_path / "nvidia-smi"
+    exe.write_text("#!/usr/bin/env python3\nimport sys, time\n"
+                   f"while True:\n    print('0, {mhz}, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, Active',"
+                   " flush=True)\n"
+                   f"    time.sleep({period_s})\n")
+    exe.chmod(0o755)
+    return str(tmp_path)
+
+
+def test_clock_sampler_region_and_short_region(tmp_path, monkeypatch):
+    """Samples come from the region only (the sampler waits for its first sample
+    before the region starts); a region shorter than the period is described by
+    the first sample after it, and says so."""
+    import os
+    import time
+    import bench
+    monkeypatch.setenv("PATH", _fake_smi(tmp_path, 0.05, 1800) + os.pathsep + os.environ["PATH"])
+    with bench.ClockSampler(0) as clk:
+        time.sleep(0.3)
+    s = clk.summary()
+    assert s["sm_mhz"] == 1800.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and s["samples"] >= 3 and "window" not in s
+    monkeypatch.setenv("PATH", _fake_smi(tmp_path, 0.3, 1500) + os.pathsep + os.environ["PATH"])
+    with bench.ClockSampler(0) as clk:
+        pass
+    s = clk.summary()
+    assert s["sm_mhz"] == 1500.0 and s["samples"] >= 1 and "window" in s
